@@ -1,0 +1,211 @@
+// Exported C ABI of libmla: argument validation, error reporting, planning and launches.
+#include "mla_internal.h"
+#include "plan_format.h"
+#include "tmap.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+namespace mla {
+
+static thread_local char g_err[512] = "";
+
+mla_status_t set_error(mla_status_t code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+mla_status_t encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                              const uint64_t* strides_bytes, const uint32_t* box,
+                              CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t d[5], s[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, s,
+                  b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static mla_status_t check_ptr(const void* p, const char* name) {
+  if (!p) return set_error(MLA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return set_error(MLA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return MLA_OK;
+}
+
+static mla_status_t check_dims(const mla_dims_t* d) {
+  if (!d) return set_error(MLA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->B < 1 || d->num_blocks < 1 || d->max_blocks_per_seq < 1)
+    return set_error(MLA_ERR_INVALID_ARG, "B, num_blocks and max_blocks_per_seq must be >= 1");
+  if (d->d_nope != 128 || d->d_rope != 64 || d->d_c != 512 || d->d_v != 128 || d->page_size != 64)
+    return set_error(MLA_ERR_UNSUPPORTED,
+                     "only d_nope=128, d_rope=64, d_c=512, d_v=128, page_size=64 are supported");
+  if (d->s_q != 1 && d->s_q != 2) return set_error(MLA_ERR_UNSUPPORTED, "s_q must be 1 or 2");
+  if (d->n_heads < 1 || d->n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
+  if (!(d->scale > 0.f) || d->scale != d->scale) return set_error(MLA_ERR_INVALID_ARG, "scale must be > 0");
+  if ((int64_t)d->num_blocks * 64 > INT32_MAX) return set_error(MLA_ERR_UNSUPPORTED, "pool too large");
+  if ((int64_t)d->B * d->s_q > 65536) return set_error(MLA_ERR_UNSUPPORTED, "more than 65536 query rows");
+  return MLA_OK;
+}
+
+static mla_status_t check_tokens(int n_tokens, int n_heads) {
+  if (n_tokens < 1 || n_tokens > 65536) return set_error(MLA_ERR_UNSUPPORTED, "n_tokens must be in [1, 65536]");
+  if (n_heads < 1 || n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
+  return MLA_OK;
+}
+
+}  // namespace mla
+
+using namespace mla;
+
+#define MLA_TRY(x)                     \
+  do {                                 \
+    mla_status_t _s = (x);             \
+    if (_s != MLA_OK) return _s;       \
+  } while (0)
+
+extern "C" {
+
+int32_t mla_version(void) { return 100; }
+
+const char* mla_last_error_string(void) { return g_err; }
+
+mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, int32_t n_tokens,
+                          int32_t n_heads, void* stream) {
+  clear_error();
+  MLA_TRY(check_tokens(n_tokens, n_heads));
+  MLA_TRY(check_ptr(q_nope, "q_nope"));
+  MLA_TRY(check_ptr(w_uk, "w_uk"));
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  return launch_absorb_q(q_nope, w_uk, q_lat, n_tokens, n_heads, stream);
+}
+
+mla_status_t mla_out_uv(const void* o_lat, const void* w_uv, void* out, int32_t n_tokens,
+                        int32_t n_heads, void* stream) {
+  clear_error();
+  MLA_TRY(check_tokens(n_tokens, n_heads));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  MLA_TRY(check_ptr(w_uv, "w_uv"));
+  MLA_TRY(check_ptr(out, "out"));
+  return launch_out_uv(o_lat, w_uv, out, n_tokens, n_heads, stream);
+}
+
+mla_status_t mla_max_clusters(int32_t* num_clusters) {
+  clear_error();
+  if (!num_clusters) return set_error(MLA_ERR_INVALID_ARG, "num_clusters is NULL");
+  return decode_max_clusters(num_clusters);
+}
+
+mla_status_t mla_plan_size(const mla_dims_t* dims, int32_t num_clusters, size_t* plan_bytes,
+                           size_t* o_part_bytes, size_t* lse_part_bytes) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  if (num_clusters < 1 || num_clusters > 4096)
+    return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
+  const int32_t N = dims->B * dims->s_q;
+  const int64_t slots = plan_slots_upper_bound(num_clusters, N);
+  if (plan_bytes) *plan_bytes = (size_t)plan_words_upper_bound(num_clusters, N) * 4;
+  if (o_part_bytes) *o_part_bytes = (size_t)slots * dims->n_heads * 512 * 4;
+  if (lse_part_bytes) *lse_part_bytes = (size_t)slots * dims->n_heads * 4;
+  return MLA_OK;
+}
+
+mla_status_t mla_plan(const mla_dims_t* dims, const int32_t* seq_lens_host, int32_t num_clusters,
+                      void* plan_host, size_t plan_bytes, int32_t* num_slots) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  if (!seq_lens_host || !plan_host) return set_error(MLA_ERR_INVALID_ARG, "NULL host buffer");
+  if (num_clusters < 1 || num_clusters > 4096)
+    return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
+  if ((reinterpret_cast<uintptr_t>(plan_host) & 3u) != 0)
+    return set_error(MLA_ERR_INVALID_ARG, "plan_host must be 4-byte aligned");
+  return build_plan(*dims, seq_lens_host, num_clusters, static_cast<int32_t*>(plan_host),
+                    (int64_t)(plan_bytes / 4), num_slots);
+}
+
+mla_status_t mla_decode_attn(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                             const void* kv_pool, const int32_t* block_table,
+                             const int32_t* seq_lens, const void* plan_dev, int32_t num_clusters,
+                             float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                             int32_t* status, void* stream) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  MLA_TRY(check_ptr(q_rope, "q_rope"));
+  MLA_TRY(check_ptr(kv_pool, "kv_pool"));
+  MLA_TRY(check_ptr(block_table, "block_table"));
+  MLA_TRY(check_ptr(seq_lens, "seq_lens"));
+  MLA_TRY(check_ptr(plan_dev, "plan_dev"));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  if (num_clusters < 1 || num_clusters > 4096)
+    return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
+  // o_part / lse_part may be NULL only when the plan splits no row; the kernel
+  // checks slots against the plan, the host cannot see the device plan here.
+  if ((o_part && !aligned16(o_part)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
+    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 16-byte aligned, lse_part 4-byte aligned");
+  return launch_decode_attn(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens,
+                            static_cast<const int32_t*>(plan_dev), num_clusters, o_part, lse_part,
+                            o_lat, lse_out, status, stream);
+}
+
+mla_status_t mla_combine(const mla_dims_t* dims, const void* plan_dev, const float* o_part,
+                         const float* lse_part, void* o_lat, float* lse_out, void* stream) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  MLA_TRY(check_ptr(plan_dev, "plan_dev"));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  if (!o_part || !lse_part) return set_error(MLA_ERR_INVALID_ARG, "o_part / lse_part is NULL");
+  return launch_combine(*dims, static_cast<const int32_t*>(plan_dev), dims->B * dims->s_q, o_part,
+                        lse_part, o_lat, lse_out, stream);
+}
+
+mla_status_t mla_debug_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
+                                    int32_t n_pages, int32_t max_blocks_per_seq, int32_t num_blocks,
+                                    void* out, int32_t* status, void* stream) {
+  clear_error();
+  MLA_TRY(check_ptr(kv_pool, "kv_pool"));
+  MLA_TRY(check_ptr(block_table, "block_table"));
+  MLA_TRY(check_ptr(out, "out"));
+  if (b < 0 || n_pages < 0 || n_pages > max_blocks_per_seq || num_blocks < 1)
+    return set_error(MLA_ERR_INVALID_ARG, "bad gather arguments");
+  return launch_gather_pages(kv_pool, block_table, b, n_pages, max_blocks_per_seq, num_blocks, out,
+                             status, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// Log-sum-exp merge of split-KV pieces, and a bit-exact page-gather check kernel.
+//
+// A row cut into pieces i = 1..m by the planner has per-piece normalised
+// outputs O_i and natural-log LSEs lse_i.  Softmax over the union of the
+// pieces' keys is
+//   L = log sum_i exp(lse_i),   o = sum_i exp(lse_i - L) O_i,
+// the identity the oracle's split-merge pin checks.  HBM-bound: one warp per
+// (row, head) reads m x 512 fp32 with 16-byte loads and writes 512 bf16.
+#include "mla_internal.h"
+#include "plan_format.h"
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+namespace mla {
+namespace {
+
+
+__global__ void __launch_bounds__(128)
+mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o_part,
+                   const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o_lat,
+                   float* __restrict__ lse_out, int n_heads) {
+  const int n = blockIdx.x;
+  const int h = blockIdx.y * 4 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (h >= n_heads) return;
+  const int32_t* rs = plan + plan[kHdrOffRows];
+  const int s0 = rs[n], s1 = rs[n + 1];
+  if (s1 <= s0) return;   // row written whole by the attention kernel
+
+  float lmax = -CUDART_INF_F;
+  for (int s = s0; s < s1; ++s) lmax = fmaxf(lmax, lse_part[(size_t)s * n_heads + h]);
+  float z = 0.f;
+  for (int s = s0; s < s1; ++s) {
+    const float l = lse_part[(size_t)s * n_heads + h];
+    z += (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax);
+  }
+  const float inv_z = z > 0.f ? 1.f / z : 0.f;
+
+  float4 acc[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = s0; s < s1; ++s) {
+    const float l = lse_part[(size_t)s * n_heads + h];
+    const float wgt = (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax) * inv_z;
+    const float4* src = reinterpret_cast<const float4*>(o_part + ((size_t)s * n_heads + h) * 512);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = __ldg(src + k * 32 + lane);
+      acc[k].x += wgt * v.x; acc[k].y += wgt * v.y; acc[k].z += wgt * v.z; acc[k].w += wgt * v.w;
+    }
+  }
+  __nv_bfloat16* dst = o_lat + ((size_t)n * n_heads + h) * 512;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(acc[k].x, acc[k].y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(acc[k].z, acc[k].w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&a);
+    u.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(dst + (k * 32 + lane) * 4) = u;
+  }
+  if (lse_out && lane == 0) lse_out[(size_t)n * n_heads + h] = z > 0.f ? lmax + __logf(z) : -CUDART_INF_F;
+}
+
+__global__ void mla_gather_pages_kernel(const uint4* __restrict__ pool, const int32_t* __restrict__ bt,
+                                        int b, int n_pages, int max_blocks, int num_blocks,
+                                        uint4* __restrict__ out, int32_t* status) {
+  constexpr int kPageVec = 64 * 576 * 2 / 16;   // 16-byte words per page
+  const int pg = blockIdx.x;
+  if (pg >= n_pages) return;
+  const int blk = bt[(size_t)b * max_blocks + pg];
+  const bool ok = blk >= 0 && blk < num_blocks;
+  if (!ok && threadIdx.x == 0 && status) atomicOr(status, MLA_STATUS_BAD_BLOCK);
+  for (int i = threadIdx.x; i < kPageVec; i += blockDim.x)
+    out[(size_t)pg * kPageVec + i] = ok ? pool[(size_t)blk * kPageVec + i] : make_uint4(0, 0, 0, 0);
+}
+
+}  // namespace
+
+mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,
+                            const float* o_part, const float* lse_part, void* o_lat,
+                            float* lse_out, void* stream) {
+  dim3 grid(n_rows, (d.n_heads + 3) / 4);
+  mla_combine_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse_out, d.n_heads);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
+                                 int32_t n_pages, int32_t max_blocks, int32_t num_blocks, void* out,
+                                 int32_t* status, void* stream) {
+  if (n_pages <= 0) return MLA_OK;
+  mla_gather_pages_kernel<<<n_pages, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(kv_pool), block_table, b, n_pages, max_blocks, num_blocks,
+      static_cast<uint4*>(out), status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "gather launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+}  // namespace mla

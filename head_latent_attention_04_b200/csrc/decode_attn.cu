@@ -1,0 +1,524 @@
+// Absorbed MLA decode attention on sm_100a (tcgen05 + TMEM + TMA + 2-CTA clusters).
+//
+// What it computes, per query row (token n, head h), over keys t < kv_len:
+//   logit_t = scale * (q_lat[n,h,:] . c_KV[t,:] + q_rope[n,h,:] . k_rope[t,:])
+//   o_lat[n,h,:] = sum_t softmax(logit)_t c_KV[t,:]
+// i.e. Step 3 of order 2 of the first absorption (term 2bhstk) plus the
+// RoPE-MQA score, then Step 1 of order 2 of the second absorption (2bhskt),
+// in the notation of "MLA Matrix Absorption Analysis" (sections 2.2, 3.2).  The
+// RoPE term of the izhida.com answer is the extra 64-wide shared key.
+//
+// Why this shape on B200.  The 128 heads of a query share one cache stream,
+// so S = [q_lat | q_rope] [c_KV | k_rope]^T (M = 128 heads, N = 64 keys,
+// K = 576) and O += P c_KV (M = 128, N = 512, K = 64) are dense contractions
+// for the tensor cores.  O for 128 heads x 512 latent columns in fp32 is
+// exactly one SM's 512 TMEM columns, leaving no room for S.  So a cluster of
+// two CTAs splits the latent dimension: CTA r owns latent columns
+// [256r, 256r + 256) and RoPE columns [32r, 32r + 32).  Each CTA stages only
+// its half of every cache row (each byte is read from HBM once), computes a
+// partial score over its 288 columns, and the two partial scores are
+// exchanged through distributed shared memory and summed (fp32 addition is
+// commutative, so both CTAs hold bit-identical scores and take identical
+// softmax decisions).  Each CTA then accumulates its 256 output columns.
+//
+// TMEM (512 columns): O [0,256) fp32, S double buffer [256,384) fp32,
+// q_lat half [384,512) as the bf16 A operand of the QK product.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
+// TMEM owner, warps 2-5 = softmax / correction / epilogue (thread = one head
+// row, i.e. one TMEM lane).  The grid is persistent: one cluster per SM pair,
+// each walking the contiguous list of (row, page range) items the host plan
+// gives it.  Every wait is bounded (ptx::kWaitLimitNs); on expiry the CTA sets
+// MLA_STATUS_TIMEOUT and unwinds without trapping.
+#include "mla_internal.h"
+#include "plan_format.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+namespace mla {
+namespace {
+
+using namespace ptx;
+
+constexpr int kPage = 64;
+constexpr int kRows = 128;
+constexpr int kStages = 4;
+constexpr int kChunkBytes = kPage * 128;                     // 64 keys x 64 latent cols (SW128)
+constexpr int kRopeBytes = kPage * 64;                       // 64 keys x 32 rope cols (SW64)
+constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;    // 36 KB: half a page
+constexpr int kQRopeBytes = kRows * 64;                      // 128 rows x 32 rope cols (SW64)
+constexpr int kPBytes = kRows * 128;                         // 128 rows x 64 keys bf16 (SW128)
+constexpr int kXRow = 64 * 4 + 16;                           // padded fp32 score row
+constexpr int kXBytes = kRows * kXRow;
+
+constexpr int kOffKV = 0;
+constexpr int kOffQRope = kOffKV + kStages * kStageBytes;
+constexpr int kOffP = kOffQRope + kQRopeBytes;
+constexpr int kOffX = kOffP + 2 * kPBytes;
+constexpr int kOffBar = kOffX + kXBytes;
+constexpr int kNumBars = 2 * kStages + 16;
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384, kTmemCols = 512;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
+
+struct DecodeParams {
+  const __nv_bfloat16* q_lat;   // [N][H][512]
+  const int32_t* block_table;   // [B][max_blocks]
+  const int32_t* seq_lens;      // [B]
+  const int32_t* plan;
+  float* o_part;                // [slots][H][512]
+  float* lse_part;              // [slots][H]
+  __nv_bfloat16* o_lat;         // [N][H][512]
+  float* lse_out;               // [N][H] or null
+  int32_t* status;
+  int n_heads, max_blocks, num_blocks, s_q, causal, B, n_rows, num_clusters;
+  float scale_log2;             // scale * log2(e)
+};
+
+struct Bars {
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], s_free[2], p_full[2], p_free[2];
+  uint64_t o_full, o_free, x_full, x_free, mma_done, pad;
+};
+static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
+
+__device__ __forceinline__ void report(int32_t* status, int bits) {
+  if (status) atomicOr(status, bits);
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+}
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort));
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rope,
+                  const __grid_constant__ CUtensorMap tm_qrope, const DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_kv = smem + kOffKV;
+  uint8_t* s_qrope = smem + kOffQRope;
+  uint8_t* s_p = smem + kOffP;
+  uint8_t* s_x = smem + kOffX;
+  Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + sizeof(Bars));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
+  const int cid = (int)cluster_id_x();
+
+  // The plan must match the launch (uniform over the grid).
+  const int32_t* plan = p.plan;
+  const bool plan_ok = plan[kHdrMagic] == kPlanMagic && plan[kHdrNumClusters] == p.num_clusters &&
+                       plan[kHdrNumRows] == p.n_rows && plan[kHdrHeads] == p.n_heads;
+  const int32_t* items = plan + plan[kHdrOffItems];
+  const int it_begin = plan_ok ? plan[plan[kHdrOffCluster] + cid] : 0;
+  const int it_end = plan_ok ? plan[plan[kHdrOffCluster] + cid + 1] : 0;
+  if (!plan_ok && threadIdx.x == 0 && rank == 0 && cid == 0) report(p.status, MLA_STATUS_BAD_SEQLEN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->q_full, 1 + kRows);
+    mbar_init(&bars->q_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->s_free[b], kRows);
+      mbar_init(&bars->p_full[b], kRows);
+      mbar_init(&bars->p_free[b], 1);
+    }
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_free, kRows);
+    mbar_init(&bars->x_full, kRows);
+    mbar_init(&bars->x_free, kRows);
+    mbar_init(&bars->mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_kv);
+    prefetch_tmap(&tm_rope);
+    prefetch_tmap(&tm_qrope);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // peer barriers initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int g = 0;
+      for (int it = it_begin; it < it_end && !*abort_flag; ++it) {
+        const int32_t* w = items + (size_t)it * kItemWords;
+        const int b = w[kItB], row = w[kItRow];
+        const int ii = it - it_begin;
+        if (ii > 0 && !mbar_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto producer_fail;
+        mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
+        tma_load_3d(s_qrope, &tm_qrope, &bars->q_full, 32 * rank, 0, row);
+        for (int pg = w[kItPageBegin]; pg < w[kItPageEnd]; ++pg, ++g) {
+          const int s = g % kStages;
+          if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, abort_flag))
+            goto producer_fail;
+          int blk = p.block_table[(size_t)b * p.max_blocks + pg];
+          if (blk < 0 || blk >= p.num_blocks) {
+            report(p.status, MLA_STATUS_BAD_BLOCK);
+            blk = 0;
+          }
+          uint8_t* st = s_kv + s * kStageBytes;
+          mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tma_load_2d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, blk * kPage);
+          tma_load_2d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, blk * kPage);
+        }
+      }
+      goto producer_drain;
+    producer_fail:
+      *abort_flag = 1;
+      report(p.status, MLA_STATUS_TIMEOUT);
+    producer_drain:
+      // every issued load must land before the CTA may exit
+      for (int k = g - 1; k >= 0 && k >= g - kStages; --k)
+        mbar_wait(&bars->kv_full[k % kStages], (k / kStages) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
+      const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+      const uint32_t kv0 = smem_u32(s_kv), qr0 = smem_u32(s_qrope), p0 = smem_u32(s_p);
+      int g = 0;
+      bool ok = true;
+      auto issue_qk = [&](int gq) -> bool {
+        const int s = gq % kStages, b = gq & 1;
+        if (!mbar_wait(&bars->kv_full[s], (gq / kStages) & 1, abort_flag)) return false;
+        if (gq >= 2 && !mbar_wait(&bars->s_free[b], ((gq >> 1) - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + kTmemS + 64 * b;
+        const uint32_t st = kv0 + s * kStageBytes;
+#pragma unroll
+        for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16
+          mma_ts(d, tmem + kTmemQ + 8 * t,
+                 sdesc(st + (t >> 2) * kChunkBytes + (t & 3) * 32, 16, 1024, kSwizzle128B), idesc_qk,
+                 t != 0);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)    // RoPE half: K = 32
+          mma_ss(d, sdesc(qr0 + t * 32, 16, 512, kSwizzle64B),
+                 sdesc(st + 4 * kChunkBytes + t * 32, 16, 512, kSwizzle64B), idesc_qk, 1);
+        mma_commit(&bars->s_full[b]);
+        return true;
+      };
+      for (int it = it_begin; it < it_end && ok; ++it) {
+        const int32_t* w = items + (size_t)it * kItemWords;
+        const int n = w[kItPageEnd] - w[kItPageBegin];
+        const int ii = it - it_begin;
+        if (!mbar_wait(&bars->q_full, ii & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (!issue_qk(g)) { ok = false; break; }
+        if (n == 1) mma_commit(&bars->q_empty);
+        for (int j = 0; j < n; ++j) {
+          if (j + 1 < n) {
+            if (!issue_qk(g + j + 1)) { ok = false; break; }
+            if (j + 2 == n) mma_commit(&bars->q_empty);
+          }
+          const int gj = g + j, b = gj & 1, s = gj % kStages;
+          if (!mbar_wait(&bars->p_full[b], (gj >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = kv0 + s * kStageBytes, pb = p0 + b * kPBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16
+            mma_ss(tmem + kTmemO, sdesc(pb + kk * 32, 16, 1024, kSwizzle128B),
+                   sdesc(st + kk * 2048, kChunkBytes, 1024, kSwizzle128B), idesc_pv, (j | kk) != 0);
+          mma_commit(&bars->p_free[b]);
+          mma_commit(&bars->kv_empty[s]);
+          mma_commit(&bars->o_full);
+        }
+        g += n;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(p.status, MLA_STATUS_TIMEOUT);
+      }
+      mma_commit(&bars->mma_done);
+      mbar_wait(&bars->mma_done, 0, nullptr);   // no MMA may still write TMEM at dealloc
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int quarter = warp & 3;                 // TMEM lanes this warp may touch
+    const int r = quarter * 32 + lane;            // head row = TMEM lane
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t x_row = smem_u32(s_x) + r * kXRow;
+    const uint32_t x_row_peer = mapa(x_row, peer);
+    const uint32_t x_full_peer = mapa(smem_u32(&bars->x_full), peer);
+    const uint32_t x_free_peer = mapa(smem_u32(&bars->x_free), peer);
+    const float* xr = reinterpret_cast<const float*>(s_x + r * kXRow);
+    uint8_t* prow0 = s_p + r * 128;
+    int g = 0;
+    for (int it = it_begin; it < it_end; ++it) {
+      const int32_t* w = items + (size_t)it * kItemWords;
+      const int row = w[kItRow], pb = w[kItPageBegin], n = w[kItPageEnd] - pb;
+      const int kv_len = w[kItKvLen], slot = w[kItSlot];
+      const int ii = it - it_begin;
+
+      // q_lat half of this row -> TMEM (bf16 pairs, A operand of the QK product)
+      if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto softmax_fail;
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)row * p.n_heads + r) * 512 + 256 * rank);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            uint4 q = r < p.n_heads ? __ldg(src + c * 8 + k) : make_uint4(0, 0, 0, 0);
+            v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
+          }
+          tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->q_full);
+      }
+
+      float m_ref = -CUDART_INF_F, l_run = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const int gj = g + j, b = gj & 1;
+        float sc[64];
+        // own partial scores
+        if (!warp_wait(&bars->s_full[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
+        tc_fence_after();
+        {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + kTmemS + 64 * b, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) sc[k] = __uint_as_float(v[k]);
+          tmem_ld32(tmem + lane_addr + kTmemS + 64 * b + 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) sc[32 + k] = __uint_as_float(v[k]);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[b]);
+
+        // exchange partial scores with the peer CTA through distributed shared memory
+        if (gj >= 1 && !warp_wait_cluster(&bars->x_free, (gj - 1) & 1, abort_flag)) goto softmax_fail;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          st_cluster_v4(x_row_peer + 16 * k, sc[4 * k], sc[4 * k + 1], sc[4 * k + 2], sc[4 * k + 3]);
+        mbar_arrive_cluster(x_full_peer);
+        if (!warp_wait_cluster(&bars->x_full, gj & 1, abort_flag)) goto softmax_fail;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float4 o = *reinterpret_cast<const float4*>(xr + 4 * k);
+          sc[4 * k] += o.x; sc[4 * k + 1] += o.y; sc[4 * k + 2] += o.z; sc[4 * k + 3] += o.w;
+        }
+        mbar_arrive_cluster(x_free_peer);
+
+        // scale (log2 domain), mask keys past kv_len, running max with lazy reference
+        const int tok0 = (pb + j) * kPage;
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          sc[k] = (tok0 + k < kv_len) ? sc[k] * p.scale_log2 : -CUDART_INF_F;
+          mx = fmaxf(mx, sc[k]);
+        }
+        const float m_new = fmaxf(m_ref, mx);
+        const bool move = (m_ref == -CUDART_INF_F) ? (m_new != -CUDART_INF_F)
+                                                   : (m_new > m_ref + kRescaleThreshold);
+        float alpha = 1.f;
+        if (move) {
+          alpha = (m_ref == -CUDART_INF_F) ? 0.f : exp2f(m_ref - m_new);
+          m_ref = m_new;
+        }
+        const float base = (m_ref == -CUDART_INF_F) ? 0.f : m_ref;
+        uint32_t pk[32];
+        float psum = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float e0 = exp2f(sc[2 * k] - base), e1 = exp2f(sc[2 * k + 1] - base);
+          pk[k] = pack_bf16(e0, e1);
+          const __nv_bfloat162 rb = *reinterpret_cast<__nv_bfloat162*>(&pk[k]);
+          psum += __bfloat162float(rb.x) + __bfloat162float(rb.y);
+        }
+        l_run = l_run * alpha + psum;
+
+        // P buffer b is free once the PV product two pages back has completed
+        if (gj >= 2 && !warp_wait(&bars->p_free[b], ((gj >> 1) - 1) & 1, abort_flag)) goto softmax_fail;
+        // rescale O in TMEM when this row's reference max moved (rare after the first page)
+        if (__any_sync(0xffffffffu, move && j > 0)) {
+          if (!warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
+          tc_fence_after();
+          const float a = (move && j > 0) ? alpha : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_addr + kTmemO + 32 * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * a);
+            tmem_st32(tmem + lane_addr + kTmemO + 32 * c, v);
+          }
+          tmem_st_wait();
+        }
+        // P row (64 keys, bf16) into the 128B-swizzled K-major A tile
+        {
+          uint8_t* prow = prow0 + b * kPBytes;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(prow + ((k ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[b]);
+      }
+
+      // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot
+      {
+        const int gl = g + n - 1;
+        if (!warp_wait(&bars->o_full, gl & 1, abort_flag)) goto softmax_fail;
+        tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        const bool valid = r < p.n_heads;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + kTmemO + 32 * c, v);
+          tmem_ld_wait();
+          if (!valid) continue;
+          const int col = 256 * rank + 32 * c;
+          if (slot < 0) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o_lat + ((size_t)row * p.n_heads + r) * 512 + col);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              dst[k] = make_uint4(pack_bf16(__uint_as_float(v[8 * k]) * inv_l, __uint_as_float(v[8 * k + 1]) * inv_l),
+                                  pack_bf16(__uint_as_float(v[8 * k + 2]) * inv_l, __uint_as_float(v[8 * k + 3]) * inv_l),
+                                  pack_bf16(__uint_as_float(v[8 * k + 4]) * inv_l, __uint_as_float(v[8 * k + 5]) * inv_l),
+                                  pack_bf16(__uint_as_float(v[8 * k + 6]) * inv_l, __uint_as_float(v[8 * k + 7]) * inv_l));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.o_part + ((size_t)slot * p.n_heads + r) * 512 + col);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              dst[k] = make_float4(__uint_as_float(v[4 * k]) * inv_l, __uint_as_float(v[4 * k + 1]) * inv_l,
+                                   __uint_as_float(v[4 * k + 2]) * inv_l, __uint_as_float(v[4 * k + 3]) * inv_l);
+          }
+        }
+        if (valid && rank == 0) {
+          const float lse = (l_run > 0.f) ? (m_ref + __log2f(l_run)) * kLn2 : -CUDART_INF_F;
+          if (slot >= 0) p.lse_part[(size_t)slot * p.n_heads + r] = lse;
+          else if (p.lse_out) p.lse_out[(size_t)row * p.n_heads + r] = lse;
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->o_free);
+      }
+      g += n;
+    }
+    goto softmax_done;
+  softmax_fail:
+    *abort_flag = 1;
+    if (lane == 0) report(p.status, MLA_STATUS_TIMEOUT);
+  softmax_done:;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  cluster_sync();   // no CTA leaves while its peer may still write into its shared memory
+}
+
+}  // namespace
+
+mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+                                const void* kv_pool, const int32_t* block_table,
+                                const int32_t* seq_lens, const int32_t* plan_dev,
+                                int32_t num_clusters, float* o_part, float* lse_part,
+                                void* o_lat, float* lse_out, int32_t* status, void* stream) {
+  CUtensorMap tm_kv, tm_rope, tm_q;
+  const uint64_t pdims[2] = {576, (uint64_t)d.num_blocks * kPage};
+  const uint64_t pstr[1] = {576 * 2};
+  const uint32_t box_kv[2] = {64, kPage};
+  const uint32_t box_rope[2] = {32, kPage};
+  mla_status_t st = encode_tmap_bf16(&tm_kv, kv_pool, 2, pdims, pstr, box_kv, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != MLA_OK) return st;
+  st = encode_tmap_bf16(&tm_rope, kv_pool, 2, pdims, pstr, box_rope, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != MLA_OK) return st;
+  const int N = d.B * d.s_q;
+  const uint64_t qdims[3] = {64, (uint64_t)d.n_heads, (uint64_t)N};
+  const uint64_t qstr[2] = {64 * 2, (uint64_t)d.n_heads * 64 * 2};
+  const uint32_t box_q[3] = {32, kRows, 1};
+  st = encode_tmap_bf16(&tm_q, q_rope, 3, qdims, qstr, box_q, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (st != MLA_OK) return st;
+
+  DecodeParams p;
+  p.q_lat = static_cast<const __nv_bfloat16*>(q_lat);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.plan = plan_dev;
+  p.o_part = o_part;
+  p.lse_part = lse_part;
+  p.o_lat = static_cast<__nv_bfloat16*>(o_lat);
+  p.lse_out = lse_out;
+  p.status = status;
+  p.n_heads = d.n_heads;
+  p.max_blocks = d.max_blocks_per_seq;
+  p.num_blocks = d.num_blocks;
+  p.s_q = d.s_q;
+  p.causal = d.causal;
+  p.B = d.B;
+  p.n_rows = N;
+  p.num_clusters = num_clusters;
+  p.scale_log2 = d.scale * 1.4426950408889634f;
+
+  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e == cudaSuccess) {
+    mla_decode_kernel<<<2 * num_clusters, 192, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tm_kv, tm_rope, tm_q, p);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t decode_max_clusters(int32_t* n) {
+  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "max clusters: %s", cudaGetErrorString(e));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int count = 0;
+  e = cudaOccupancyMaxActiveClusters(&count, mla_decode_kernel, &cfg);
+  if (e != cudaSuccess || count <= 0) {
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    count = sms / 2;
+    cudaGetLastError();
+  }
+  *n = count;
+  return MLA_OK;
+}
+
+}  // namespace mla

@@ -1,0 +1,34 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include "../../include/mla.h"
+
+#include <stdint.h>
+
+namespace mla {
+
+// Records a printf-style message in the thread-local error slot; returns `code`.
+mla_status_t set_error(mla_status_t code, const char* fmt, ...);
+void clear_error();
+
+mla_status_t build_plan(const mla_dims_t& d, const int32_t* seq_lens, int32_t num_clusters,
+                        int32_t* plan, int64_t plan_words, int32_t* num_slots_out);
+
+// Kernel launchers (defined in the .cu files); each returns MLA_OK or MLA_ERR_CUDA.
+mla_status_t launch_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, int n_tokens,
+                             int n_heads, void* stream);
+mla_status_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int n_tokens,
+                           int n_heads, void* stream);
+mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+                                const void* kv_pool, const int32_t* block_table,
+                                const int32_t* seq_lens, const int32_t* plan_dev,
+                                int32_t num_clusters, float* o_part, float* lse_part,
+                                void* o_lat, float* lse_out, int32_t* status, void* stream);
+mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,
+                            const float* o_part, const float* lse_part, void* o_lat,
+                            float* lse_out, void* stream);
+mla_status_t launch_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
+                                 int32_t n_pages, int32_t max_blocks, int32_t num_blocks, void* out,
+                                 int32_t* status, void* stream);
+mla_status_t decode_max_clusters(int32_t* n);
+
+}  // namespace mla

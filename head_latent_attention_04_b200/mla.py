@@ -1,0 +1,215 @@
+"""ctypes binding of libmla (include/mla.h): argument marshalling only.
+
+Every step of the decode path runs in the library's CUDA kernels; this module
+turns torch tensors into device pointers and the current CUDA stream into a
+cudaStream_t, and raises on error codes.  Importing it fails loudly when the
+shared library has not been built: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libmla.so is not built ({_LIB_PATH}); run "
+                      "`python -m head_latent_attention_04_b200.build`")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED = 0, 1, 2
+MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_TIMEOUT = 3, 4, 5
+STATUS_BAD_BLOCK, STATUS_TIMEOUT, STATUS_BAD_SEQLEN = 0x1, 0x2, 0x4
+EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
+           "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
+           "mla_debug_gather_pages")
+
+
+class MlaDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("s_q", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+                ("d_nope", ctypes.c_int32), ("d_rope", ctypes.c_int32), ("d_c", ctypes.c_int32),
+                ("d_v", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("max_blocks_per_seq", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("causal", ctypes.c_int32)]
+
+
+_vp, _i32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+_pdims = ctypes.POINTER(MlaDims)
+_lib.mla_version.restype = _i32
+_lib.mla_last_error_string.restype = ctypes.c_char_p
+for _name, _args in {
+    "mla_absorb_q": [_vp, _vp, _vp, _i32, _i32, _vp],
+    "mla_out_uv": [_vp, _vp, _vp, _i32, _i32, _vp],
+    "mla_max_clusters": [ctypes.POINTER(_i32)],
+    "mla_plan_size": [_pdims, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
+    "mla_plan": [_pdims, _vp, _i32, _vp, _sz, ctypes.POINTER(_i32)],
+    "mla_decode_attn": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
+    "mla_combine": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp],
+    "mla_debug_gather_pages": [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+}.items():
+    getattr(_lib, _name).argtypes = _args
+    getattr(_lib, _name).restype = _i32
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = _lib.mla_last_error_string().decode(errors="replace")
+        super().__init__(f"{where}: status {code}: {msg}")
+
+
+def _check(code: int, where: str):
+    if code != MLA_OK:
+        raise MlaError(code, where)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def version() -> int:
+    return _lib.mla_version()
+
+
+def make_dims(B, s_q, n_heads, max_blocks, num_blocks, scale=None, causal=True) -> MlaDims:
+    if scale is None:
+        scale = 1.0 / math.sqrt(128 + 64)
+    return MlaDims(B, s_q, n_heads, 128, 64, 512, 128, 64, max_blocks, num_blocks, float(scale),
+                   1 if causal else 0)
+
+
+def max_clusters() -> int:
+    n = _i32(0)
+    _check(_lib.mla_max_clusters(ctypes.byref(n)), "mla_max_clusters")
+    return n.value
+
+
+def plan_size(dims: MlaDims, num_clusters: int):
+    pb, ob, lb = _sz(0), _sz(0), _sz(0)
+    _check(_lib.mla_plan_size(ctypes.byref(dims), num_clusters, ctypes.byref(pb), ctypes.byref(ob),
+                              ctypes.byref(lb)), "mla_plan_size")
+    return pb.value, ob.value, lb.value
+
+
+def plan(dims: MlaDims, seq_lens, num_clusters: int):
+    """Host plan as an int32 numpy array, and the number of partial slots used."""
+    pb, _, _ = plan_size(dims, num_clusters)
+    buf = np.zeros(pb // 4, dtype=np.int32)
+    sl = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    ns = _i32(0)
+    _check(_lib.mla_plan(ctypes.byref(dims), sl.ctypes.data, num_clusters, buf.ctypes.data, pb,
+                         ctypes.byref(ns)), "mla_plan")
+    return buf, ns.value
+
+
+def absorb_q(q_nope: torch.Tensor, w_uk: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    N, H, _ = q_nope.shape
+    if out is None:
+        out = torch.empty((N, H, 512), dtype=torch.bfloat16, device=q_nope.device)
+    _check(_lib.mla_absorb_q(_ptr(q_nope), _ptr(w_uk), _ptr(out), N, H, _stream(stream)), "mla_absorb_q")
+    return out
+
+
+def out_uv(o_lat: torch.Tensor, w_uv: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    N, H, _ = o_lat.shape
+    if out is None:
+        out = torch.empty((N, H, 128), dtype=torch.bfloat16, device=o_lat.device)
+    _check(_lib.mla_out_uv(_ptr(o_lat), _ptr(w_uv), _ptr(out), N, H, _stream(stream)), "mla_out_uv")
+    return out
+
+
+def decode_attn(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_dev, num_clusters,
+                o_part, lse_part, o_lat, lse_out=None, status=None, stream=None):
+    _check(_lib.mla_decode_attn(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(kv_pool),
+                                _ptr(block_table), _ptr(seq_lens), _ptr(plan_dev), num_clusters,
+                                _ptr(o_part), _ptr(lse_part), _ptr(o_lat), _ptr(lse_out),
+                                _ptr(status), _stream(stream)), "mla_decode_attn")
+
+
+def combine(dims, plan_dev, o_part, lse_part, o_lat, lse_out=None, stream=None):
+    _check(_lib.mla_combine(ctypes.byref(dims), _ptr(plan_dev), _ptr(o_part), _ptr(lse_part),
+                            _ptr(o_lat), _ptr(lse_out), _stream(stream)), "mla_combine")
+
+
+def debug_gather_pages(kv_pool, block_table, b, n_pages, max_blocks, num_blocks, out, status=None,
+                       stream=None):
+    _check(_lib.mla_debug_gather_pages(_ptr(kv_pool), _ptr(block_table), b, n_pages, max_blocks,
+                                       num_blocks, _ptr(out), _ptr(status), _stream(stream)),
+           "mla_debug_gather_pages")
+
+
+@dataclass
+class DecodeOutputs:
+    out: torch.Tensor        # bf16 [N][h][128]
+    q_lat: torch.Tensor      # bf16 [N][h][512]
+    o_lat: torch.Tensor      # bf16 [N][h][512]
+    lse: torch.Tensor        # fp32 [N][h]
+    status: torch.Tensor     # int32 [1]
+
+
+class Decoder:
+    """One decode batch shape: plan, workspace and output buffers made once, then
+    ``run()`` enqueues absorb -> attention -> combine -> out_uv on the stream.
+
+    Buffers are allocated here by torch (the library allocates nothing).
+    """
+
+    def __init__(self, seq_lens, s_q: int, n_heads: int, max_blocks: int, num_blocks: int,
+                 device="cuda", scale=None, causal=True, num_clusters: int | None = None):
+        self.seq_lens_host = np.asarray(seq_lens, dtype=np.int32)
+        self.B = len(self.seq_lens_host)
+        self.s_q, self.H = s_q, n_heads
+        self.N = self.B * s_q
+        self.dims = make_dims(self.B, s_q, n_heads, max_blocks, num_blocks, scale, causal)
+        self.num_clusters = num_clusters or max_clusters()
+        self.plan_host, self.num_slots = plan(self.dims, self.seq_lens_host, self.num_clusters)
+        dev = torch.device(device)
+        self.plan_dev = torch.from_numpy(self.plan_host).to(dev)
+        self.seq_lens_dev = torch.from_numpy(self.seq_lens_host).to(dev)
+        slots = max(self.num_slots, 1)
+        self.o_part = torch.empty((slots, n_heads, 512), dtype=torch.float32, device=dev)
+        self.lse_part = torch.empty((slots, n_heads), dtype=torch.float32, device=dev)
+        self.q_lat = torch.empty((self.N, n_heads, 512), dtype=torch.bfloat16, device=dev)
+        self.o_lat = torch.empty((self.N, n_heads, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.N, n_heads), dtype=torch.float32, device=dev)
+        self.out = torch.empty((self.N, n_heads, 128), dtype=torch.bfloat16, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def run(self, q_nope, q_rope, kv_pool, block_table, w_uk, w_uv, stream=None) -> DecodeOutputs:
+        absorb_q(q_nope, w_uk, self.q_lat, stream)
+        decode_attn(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev,
+                    self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
+                    self.lse, self.status, stream)
+        if self.num_slots > 0:
+            combine(self.dims, self.plan_dev, self.o_part, self.lse_part, self.o_lat, self.lse, stream)
+        out_uv(self.o_lat, w_uv, self.out, stream)
+        return DecodeOutputs(self.out, self.q_lat, self.o_lat, self.lse, self.status)
+
+    @property
+    def launches_per_step(self) -> int:
+        return 4 if self.num_slots > 0 else 3
+
+
+def decode(q_nope, q_rope, kv_pool, block_table, seq_lens, w_uk, w_uv, s_q=1, scale=None,
+           causal=True, num_clusters=None) -> DecodeOutputs:
+    """One-shot absorbed MLA decode on device tensors (see ``Decoder``)."""
+    bt = block_table if isinstance(block_table, torch.Tensor) else torch.as_tensor(block_table)
+    bt = bt.to(device=kv_pool.device, dtype=torch.int32).contiguous()
+    sl = seq_lens.cpu().numpy() if isinstance(seq_lens, torch.Tensor) else np.asarray(seq_lens)
+    d = Decoder(sl, s_q, q_nope.shape[1], bt.shape[1], kv_pool.shape[0], kv_pool.device, scale,
+                causal, num_clusters)
+    return d.run(q_nope, q_rope, kv_pool, bt, w_uk, w_uv)

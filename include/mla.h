@@ -1,0 +1,176 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) absorbed MLA decode library (libmla).
+ *
+ * The library computes one decode step of DeepSeek-V2/V3 Multi-head Latent
+ * Attention (MLA) in the absorbed evaluation order ("order 2") of the MLA
+ * matrix-absorption notes (wkq9411.github.io, "MLA Matrix Absorption
+ * Analysis", section 2.2 for the logits and section 3.2 for the output):
+ *
+ *   q_lat[n,h,:] = sum_d q_nope[n,h,d] * W_UK[:,h,d]                mla_absorb_q
+ *   logit[n,h,t] = scale * (q_lat[n,h].c_KV[t] + q_rope[n,h].k_rope[t])
+ *   p = softmax_t(logit), o_lat[n,h,:] = sum_t p[t] c_KV[t]          mla_decode_attn
+ *                                                                   (+ mla_combine)
+ *   out[n,h,:]   = sum_k o_lat[n,h,k] * W_UV[k,h,:]                  mla_out_uv
+ *
+ * K = W_UK c_KV and V = W_UV c_KV are never formed, nor are W_UQ^T W_UK or
+ * W_O W_UV.  The RoPE key is the extra multi-query term of the izhida.com
+ * answer "How is DeepSeek-V2's inference cost computed?": one 64-wide
+ * post-rotation key per token, shared by all heads, whose score is added.
+ *
+ * Conventions (every entry point):
+ *   - bf16 is IEEE bfloat16 stored as uint16; fp32 is IEEE float.
+ *   - All tensor arguments are CALLER-OWNED DEVICE pointers (plan_host and
+ *     seq_lens_host excepted), contiguous row-major, 16-byte aligned.  The
+ *     library never allocates, frees or retains device memory.
+ *   - `stream` is a cudaStream_t (passed as void*); every device call is
+ *     asynchronous on it.  Host-side validation happens before any launch.
+ *   - Return value: MLA_OK or an error code; mla_last_error_string() gives a
+ *     thread-local message for the last failing call.  Nothing aborts,
+ *     throws or traps across this boundary.
+ *   - Device-detected faults (a block id outside [0, num_blocks), a wait
+ *     that ran past its time limit) set bits of the optional int32 *status
+ *     word (atomic OR) and skip or substitute the affected work; they never
+ *     trap.  Pass NULL to skip status reporting.
+ *
+ * Shapes: n_tokens N = B * s_q query rows; row n = b * s_q + i.
+ * Supported: d_nope = 128, d_rope = 64, d_c = 512, d_v = 128, page_size = 64,
+ * s_q in {1, 2}, 1 <= n_heads <= 128.  Other shapes return MLA_ERR_UNSUPPORTED.
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,        /* null/misaligned pointer, bad size, inconsistent plan */
+  MLA_ERR_UNSUPPORTED = 2,        /* shape outside the supported set */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3,
+  MLA_ERR_CUDA = 4,               /* a CUDA runtime call failed (message has the CUDA error) */
+  MLA_ERR_TIMEOUT = 5
+} mla_status_t;
+
+/* Bits set in the device status word. */
+#define MLA_STATUS_BAD_BLOCK   0x1   /* block_table entry outside [0, num_blocks): block 0 used */
+#define MLA_STATUS_TIMEOUT     0x2   /* a bounded device wait expired; outputs are invalid */
+#define MLA_STATUS_BAD_SEQLEN  0x4   /* device seq_lens disagree with the plan */
+
+/* Problem dimensions of one decode batch. */
+typedef struct {
+  int32_t B;                  /* sequences */
+  int32_t s_q;                /* new query tokens per sequence (1, or 2 for MTP) */
+  int32_t n_heads;            /* h */
+  int32_t d_nope;             /* 128 */
+  int32_t d_rope;             /* 64 */
+  int32_t d_c;                /* 512 (latent width of c_KV) */
+  int32_t d_v;                /* 128 */
+  int32_t page_size;          /* 64 tokens per cache block */
+  int32_t max_blocks_per_seq; /* columns of block_table */
+  int32_t num_blocks;         /* blocks in the cache pool */
+  float scale;                /* softmax scale, e.g. 1/sqrt(d_nope + d_rope) */
+  int32_t causal;             /* s_q == 2: 1 = query i attends t <= T - s_q + i; 0 = all T */
+} mla_dims_t;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int32_t mla_version(void);
+
+/* Thread-local message of the last failing call on this thread ("" if none). */
+const char* mla_last_error_string(void);
+
+/*
+ * mla_absorb_q -- first absorption, order 2, Step 2 of the notes' section 2.2:
+ * the per-head contraction q_lat = q_nope^T W_UK (term 2bshkd of FLOPs_order2).
+ *   q_nope  bf16 [n_tokens][n_heads][128]   (device, read)
+ *   w_uk    bf16 [512][n_heads][128]        (device, read; (k, h, d) as in section 2.1)
+ *   q_lat   bf16 [n_tokens][n_heads][512]   (device, written; fp32 accumulation, RNE to bf16)
+ * 1 <= n_tokens <= 65536.
+ */
+mla_status_t mla_absorb_q(const void* q_nope, const void* w_uk, void* q_lat,
+                          int32_t n_tokens, int32_t n_heads, void* stream);
+
+/*
+ * mla_out_uv -- second absorption, order 2, Step 2 of the notes' section 3.2:
+ * out = W_UV applied per head to the latent output (term 2bhsvk of FLOPs_order2).
+ *   o_lat   bf16 [n_tokens][n_heads][512]   (device, read)
+ *   w_uv    bf16 [512][n_heads][128]        (device, read; (k, h, v) as in section 3.1)
+ *   out     bf16 [n_tokens][n_heads][128]   (device, written; fp32 accumulation)
+ */
+mla_status_t mla_out_uv(const void* o_lat, const void* w_uv, void* out,
+                        int32_t n_tokens, int32_t n_heads, void* stream);
+
+/*
+ * Split-KV planning (host only, deterministic).  The decode kernel is a
+ * persistent grid of 2-CTA clusters; each cluster walks a contiguous range of
+ * the flattened (sequence, page) work list of one query position, so a long
+ * sequence is split across clusters and a cluster can cover several short
+ * ones.  Pieces of a split row are merged by mla_combine.
+ *
+ * mla_plan_size: upper bounds for the plan (int32 words, in bytes) and for
+ *   the two workspace arrays, o_part fp32 [slots][n_heads][512] and
+ *   lse_part fp32 [slots][n_heads], for `num_clusters` clusters.
+ * mla_plan: writes the plan into caller memory `plan_host` (plan_bytes from
+ *   mla_plan_size); the caller copies it to the device unchanged.  Fails with
+ *   MLA_ERR_INVALID_ARG if some seq_lens_host[b] < s_q or > max_blocks*64.
+ *   *num_slots receives the number of partial-output slots used.
+ * mla_max_clusters: how many decode clusters the current device runs at once
+ *   (the natural `num_clusters`).
+ */
+mla_status_t mla_max_clusters(int32_t* num_clusters);
+mla_status_t mla_plan_size(const mla_dims_t* dims, int32_t num_clusters, size_t* plan_bytes,
+                           size_t* o_part_bytes, size_t* lse_part_bytes);
+mla_status_t mla_plan(const mla_dims_t* dims, const int32_t* seq_lens_host, int32_t num_clusters,
+                      void* plan_host, size_t plan_bytes, int32_t* num_slots);
+
+/*
+ * mla_decode_attn -- the attention core: scores of the absorbed query
+ * [q_lat | q_rope] against the paged [c_KV | k_rope] cache (notes section 2.2
+ * Step 3, term 2bhstk, plus the RoPE term), softmax over t, and the weighted
+ * sum of c_KV (notes section 3.2 Step 1, term 2bhskt).
+ *   q_lat        bf16 [N][n_heads][512]     (from mla_absorb_q)
+ *   q_rope       bf16 [N][n_heads][64]      (post-rotation)
+ *   kv_pool      bf16 [num_blocks][64][576] (token row = c_KV (512) | k_rope (64))
+ *   block_table  int32 [B][max_blocks_per_seq]
+ *   seq_lens     int32 [B]  T_b, counting the s_q new tokens (checked against the plan)
+ *   plan_dev     the plan from mla_plan, copied to the device
+ *   num_clusters the num_clusters the plan was built for (grid = 2 * num_clusters CTAs)
+ *   o_part       fp32 [slots][n_heads][512]   workspace (split rows)
+ *   lse_part     fp32 [slots][n_heads]        workspace
+ *   o_lat        bf16 [N][n_heads][512]       rows not split are written here
+ *   lse_out      fp32 [N][n_heads] or NULL    natural-log LSE of the scaled logits
+ *   status       int32 [1] or NULL
+ * Rows that the plan splits are completed by mla_combine.
+ */
+mla_status_t mla_decode_attn(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                             const void* kv_pool, const int32_t* block_table,
+                             const int32_t* seq_lens, const void* plan_dev, int32_t num_clusters,
+                             float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                             int32_t* status, void* stream);
+
+/*
+ * mla_combine -- log-sum-exp merge of the split pieces of each split row:
+ *   L = log sum_i exp(lse_i),  o_lat = sum_i exp(lse_i - L) * O_i.
+ * Reads o_part/lse_part written by mla_decode_attn with the same plan, writes
+ * o_lat bf16 [N][n_heads][512] and (if non-NULL) lse_out for split rows only.
+ */
+mla_status_t mla_combine(const mla_dims_t* dims, const void* plan_dev, const float* o_part, const float* lse_part, void* o_lat,
+                         float* lse_out, void* stream);
+
+/*
+ * mla_debug_gather_pages -- copies the cache rows of sequence b, in token
+ * order, through block_table into out bf16 [n_pages*64][576] (bit-exact page
+ * indexing check; not on the decode path).  Out-of-range block ids set
+ * MLA_STATUS_BAD_BLOCK and write zeros.
+ */
+mla_status_t mla_debug_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
+                                    int32_t n_pages, int32_t max_blocks_per_seq, int32_t num_blocks,
+                                    void* out, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

@@ -1,0 +1,178 @@
+"""CUDA path vs the float64 oracle, element by element, through the C ABI.
+
+Tolerance on the final output: relative Frobenius <= 5e-3 and max abs <= 2e-2
+(bf16 inputs and intermediates q_lat / P / o_lat, fp32 accumulation).  The
+intermediates get the same relative bound.  Page indexing, the plan and
+outputs under a pool permutation are compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+from head_latent_attention_04_b200 import workloads as W
+from oracle import mla_oracle as O
+from tests.gpu_helpers import check_out, oracle_all, oracle_rows, rel_fro, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def mla():
+    from head_latent_attention_04_b200 import mla as m
+    return m
+
+
+# ------------------------------------------------------------------ projections alone
+@pytest.mark.parametrize("N,H", [(1, 1), (2, 16), (37, 128), (256, 128), (300, 7)])
+def test_absorb_q_matches_oracle(mla, N, H):
+    w = W.make_workload(1, 1, H, [1], seed=N + H)
+    g = torch.Generator().manual_seed(N)
+    q = torch.randn((N, H, 128), generator=g).to(torch.bfloat16)
+    got = mla.absorb_q(q.cuda(), w.w_uk.cuda())
+    torch.cuda.synchronize()
+    want = O.contract(None, "absorb_q", "nhd,khd->nhk", q.double().numpy(), w.w_uk.double().numpy())
+    assert rel_fro(got.float().cpu().numpy(), want) < 5e-3
+
+
+@pytest.mark.parametrize("N,H", [(1, 1), (2, 16), (37, 128), (256, 128), (130, 3)])
+def test_out_uv_matches_oracle(mla, N, H):
+    w = W.make_workload(1, 1, H, [1], seed=N + 2 * H)
+    g = torch.Generator().manual_seed(N + 7)
+    o = (torch.randn((N, H, 512), generator=g) * 0.05).to(torch.bfloat16)
+    got = mla.out_uv(o.cuda(), w.w_uv.cuda())
+    torch.cuda.synchronize()
+    want = O.contract(None, "out_uv", "nhk,khv->nhv", o.double().numpy(), w.w_uv.double().numpy())
+    assert rel_fro(got.float().cpu().numpy(), want) < 5e-3
+
+
+# ------------------------------------------------------------------ page indexing
+def test_gather_pages_bit_exact(mla):
+    w = W.make_workload(3, 1, 4, [130, 64, 5], seed=4, pool="scattered:2")
+    dev = torch.device("cuda")
+    pool = w.kv_pool.to(dev)
+    bt = torch.as_tensor(w.block_table, device=dev)
+    for b in range(3):
+        n_pages = -(-int(w.seq_lens[b]) // 64)
+        out = torch.empty((n_pages * 64, 576), dtype=torch.bfloat16, device=dev)
+        mla.debug_gather_pages(pool, bt, b, n_pages, w.max_blocks, w.num_blocks, out)
+        torch.cuda.synchronize()
+        assert torch.equal(out[: int(w.seq_lens[b])].cpu(), w.cache_rows(b))
+
+
+def test_gather_bad_block_sets_status(mla):
+    w = W.make_workload(1, 1, 4, [128], seed=5)
+    dev = torch.device("cuda")
+    bt = torch.as_tensor(w.block_table, device=dev)
+    bt[0, 1] = w.num_blocks + 5
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty((128, 576), dtype=torch.bfloat16, device=dev)
+    mla.debug_gather_pages(w.kv_pool.to(dev), bt, 0, 2, w.max_blocks, w.num_blocks, out, status)
+    torch.cuda.synchronize()
+    assert status.item() & mla.STATUS_BAD_BLOCK
+    assert torch.all(out[64:].float() == 0)
+
+
+# ------------------------------------------------------------------ the whole decode path
+def _full_check(w, num_clusters=None, rel=5e-3):
+    dec, res = run_gpu(w, num_clusters)
+    assert res.status.item() == 0
+    ref = oracle_all(w)
+    check_out(res.out, ref["out"], rel=rel)
+    assert rel_fro(res.q_lat.float().cpu().numpy(), ref["q_lat"]) < 5e-3
+    assert rel_fro(res.o_lat.float().cpu().numpy(), ref["o_lat"]) < 5e-3
+    np.testing.assert_allclose(res.lse.cpu().numpy(), ref["lse"], rtol=0, atol=2e-2)
+    return dec, res
+
+
+def test_tiny_config(mla):
+    """The small preset: B=2, h=16, T=256, contiguous cache."""
+    _full_check(W.preset_workload("tiny"))
+
+
+@pytest.mark.parametrize("clusters", [1, 2, 3, 74, 148])
+def test_split_counts(mla, clusters):
+    """Same batch under plans from no split to many pieces per row (LSE merge)."""
+    w = W.make_workload(3, 1, 32, [700, 64, 1000], seed=11, pool="permuted")
+    _full_check(w, num_clusters=clusters)
+
+
+@pytest.mark.parametrize("lens", [[1], [63], [64], [65], [1, 2, 3, 127, 128, 129, 191]])
+def test_ragged_lengths(mla, lens):
+    w = W.make_workload(len(lens), 1, 128, lens, seed=sum(lens), pool="scattered:1.5")
+    _full_check(w, num_clusters=4)
+
+
+@pytest.mark.parametrize("H", [1, 16, 100, 128])
+def test_head_counts(mla, H):
+    w = W.make_workload(2, 1, H, [300, 90], seed=H, pool="permuted")
+    _full_check(w)
+
+
+@pytest.mark.parametrize("lens,clusters", [([2, 3, 65, 66, 200], 74), ([2, 3, 65, 66, 200], 3),
+                                           ([4097, 64], 9)])
+def test_mtp_causal(mla, lens, clusters):
+    """s_q = 2, causal between the two new tokens."""
+    w = W.make_workload(len(lens), 2, 128, lens, seed=len(lens) + clusters, pool="permuted")
+    _full_check(w, num_clusters=clusters)
+
+
+def test_pool_permutation_is_bit_exact(mla):
+    """Same values, different page placement, same plan -> identical bits."""
+    a = W.make_workload(4, 1, 128, [300, 1000, 64, 513], seed=21, pool="contiguous")
+    b = W.make_workload(4, 1, 128, [300, 1000, 64, 513], seed=21, pool="scattered:3")
+    _, ra = run_gpu(a, num_clusters=6)
+    oa = ra.out.clone()
+    _, rb = run_gpu(b, num_clusters=6)
+    assert torch.equal(oa, rb.out)
+
+
+def test_poison_never_leaks(mla):
+    """Pool rows past each sequence hold a huge finite value; it must not reach the output."""
+    w = W.make_workload(2, 1, 128, [65, 130], seed=31, pool="scattered:4", poison=3.0e38)
+    _full_check(w, num_clusters=3)
+
+
+def test_bad_block_id_reports_and_does_not_trap(mla):
+    w = W.make_workload(2, 1, 16, [200, 100], seed=41)
+    w.block_table[1, 0] = -7
+    dec, res = run_gpu(w, num_clusters=2)
+    assert res.status.item() & mla.STATUS_BAD_BLOCK
+    # sequence 0 is untouched by the bad id
+    ref = oracle_rows(w, 0)
+    check_out(res.out[:1], ref["out"])
+    # the context is still usable
+    _full_check(W.preset_workload("tiny"))
+
+
+def test_stale_plan_is_rejected_on_device(mla):
+    w = W.preset_workload("tiny")
+    dev = torch.device("cuda")
+    dec, _ = run_gpu(w)
+    dec.plan_dev[0] = 0    # corrupt the magic word
+    dec.status.zero_()
+    wd = w.to(dev)
+    dec.run(wd.q_nope, wd.q_rope, wd.kv_pool, torch.as_tensor(w.block_table, device=dev),
+            wd.w_uk, wd.w_uv)
+    torch.cuda.synchronize()
+    assert dec.status.item() & mla.STATUS_BAD_SEQLEN
+
+
+# ------------------------------------------------------------------ full-size presets, sampled
+def _sampled(name, n_seq=2, heads=(0, 77, 127), seed_pick=0):
+    w = W.preset_workload(name)
+    dec, res = run_gpu(w)
+    assert res.status.item() == 0
+    out = res.out.float().cpu().numpy()
+    rng = np.random.default_rng(seed_pick)
+    seqs = sorted(set(rng.choice(w.B, size=min(n_seq, w.B), replace=False).tolist()))
+    for b in seqs:
+        ref = oracle_rows(w, b, heads=list(heads))
+        got = out[b * w.s_q:(b + 1) * w.s_q][:, list(heads)]
+        check_out(got, ref["out"])
+    assert np.all(np.isfinite(out))
+    return w, dec
+
+
+@pytest.mark.parametrize("name", ["v2_4k", "varlen", "long128k", "mtp2"])
+def test_full_size_preset_sampled(mla, name):
+    _sampled(name)

@@ -1,0 +1,157 @@
+"""Host side of the C ABI (CPU only): exports, argument validation, and the split
+planner checked bit-exactly against an independent Python derivation."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from head_latent_attention_04_b200 import mla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_library_exports_every_declared_symbol():
+    header = open(os.path.join(ROOT, "include", "mla.h")).read()
+    declared = set(re.findall(r"^\s*(?:mla_status_t|int32_t|const char\*)\s+(mla_\w+)\s*\(", header, re.M))
+    assert declared == set(mla.EXPORTS)
+    lib = ctypes.CDLL(mla._LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert mla.version() >= 100
+
+
+# ------------------------------------------------------------------ independent planner
+def py_plan(seq_lens, s_q, causal, n_heads, num_clusters, page=64):
+    """Re-derivation of the documented split rule: per query position i (its own
+    group of clusters when there are at least s_q clusters), the rows' pages are
+    concatenated in sequence order and cut at floor(c * P / G)."""
+    B = len(seq_lens)
+    N = B * s_q
+    rows = []
+    for b in range(B):
+        for i in range(s_q):
+            kv = seq_lens[b] - s_q + 1 + i if causal else seq_lens[b]
+            rows.append(dict(b=b, qi=i, kv=kv, pages=-(-kv // page)))
+    groups = s_q if num_clusters >= s_q else 1
+    G = num_clusters // groups
+    pieces = []   # (cluster, row, p0, p1)
+    for g in range(groups):
+        members = [n for n in range(N) if groups == 1 or n % s_q == g]
+        P = sum(rows[n]["pages"] for n in members)
+        off = 0
+        for n in members:
+            r0, r1 = off, off + rows[n]["pages"]
+            off = r1
+            for c in range(G):
+                lo, hi = c * P // G, (c + 1) * P // G
+                a, e = max(lo, r0), min(hi, r1)
+                if a < e:
+                    pieces.append((g * G + c, n, a - r0, e - r0))
+    count = [0] * N
+    for p in pieces:
+        count[p[1]] += 1
+    slot_begin = [0] * (N + 1)
+    for n in range(N):
+        slot_begin[n + 1] = slot_begin[n] + (count[n] if count[n] > 1 else 0)
+    seen = [0] * N
+    items = []
+    for cl, n, p0, p1 in pieces:
+        k = seen[n]
+        seen[n] += 1
+        slot = slot_begin[n] + k if count[n] > 1 else -1
+        items.append((cl, [rows[n]["b"], rows[n]["qi"], p0, p1, rows[n]["kv"], slot, n, 0]))
+    items.sort(key=lambda t: t[0])          # stable: keeps row order inside a cluster
+    cl_begin = [0] * (num_clusters + 1)
+    for cl, _ in items:
+        cl_begin[cl + 1] += 1
+    for c in range(num_clusters):
+        cl_begin[c + 1] += cl_begin[c]
+    return cl_begin, [w for _, w in items], slot_begin
+
+
+def _unpack(buf):
+    off_c, off_i, off_r = buf[8], buf[9], buf[10]
+    C, I, N = buf[1], buf[2], buf[4]
+    return (list(buf[off_c:off_c + C + 1]),
+            [list(buf[off_i + 8 * k: off_i + 8 * k + 8]) for k in range(I)],
+            list(buf[off_r:off_r + N + 1]))
+
+
+@pytest.mark.parametrize("case", [
+    dict(lens=[4096] * 32, s_q=1, H=128, C=74),
+    dict(lens=[256, 256], s_q=1, H=16, C=74),
+    dict(lens=[131072] * 4, s_q=1, H=128, C=74),
+    dict(lens=[1, 64, 65, 127, 128, 129, 5000], s_q=1, H=8, C=5),
+    dict(lens=[2, 3, 64, 65, 66, 4097, 130], s_q=2, H=128, C=74),
+    dict(lens=[2, 3, 64, 65, 66, 4097, 130], s_q=2, H=128, C=1),
+    dict(lens=[77, 9000, 300], s_q=2, H=64, C=7),
+    dict(lens=[100], s_q=1, H=1, C=3),
+])
+def test_plan_bit_exact(case):
+    dims = mla.make_dims(len(case["lens"]), case["s_q"], case["H"], max(-(-t // 64) for t in case["lens"]),
+                         10 ** 6)
+    buf, ns = mla.plan(dims, case["lens"], case["C"])
+    assert buf[0] == 0x314C414D and buf[1] == case["C"]
+    cl, items, rows = _unpack(buf)
+    ecl, eitems, erows = py_plan(case["lens"], case["s_q"], True, case["H"], case["C"])
+    assert cl == ecl and items == eitems and rows == erows
+    assert ns == erows[-1] == buf[3]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_plan_random_covers_every_page_once(seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 40))
+    s_q = int(rng.integers(1, 3))
+    lens = rng.integers(s_q, 20000, size=B).tolist()
+    C = int(rng.integers(1, 200))
+    dims = mla.make_dims(B, s_q, 128, max(-(-t // 64) for t in lens), 10 ** 6)
+    buf, ns = mla.plan(dims, lens, C)
+    cl, items, rows = _unpack(buf)
+    assert (cl, items, rows) == py_plan(lens, s_q, True, 128, C)
+    covered = {}
+    for w in items:
+        b, qi, p0, p1, kv, slot, n = w[:7]
+        assert n == b * s_q + qi and 0 <= p0 < p1 <= -(-kv // 64)
+        for p in range(p0, p1):
+            assert (n, p) not in covered
+            covered[(n, p)] = True
+    for n in range(B * s_q):
+        b, qi = divmod(n, s_q)
+        kv = lens[b] - s_q + 1 + qi
+        assert all((n, p) in covered for p in range(-(-kv // 64)))
+    pb, ob, lb = mla.plan_size(dims, C)
+    assert buf[11] * 4 <= pb and ns * 128 * 512 * 4 <= ob and ns * 128 * 4 <= lb
+
+
+# ------------------------------------------------------------------ validation (no GPU needed)
+def test_invalid_arguments_return_codes():
+    good = mla.make_dims(2, 1, 16, 4, 8)
+    for field, val, code in [("d_c", 256, mla.MLA_ERR_UNSUPPORTED), ("s_q", 3, mla.MLA_ERR_UNSUPPORTED),
+                             ("n_heads", 129, mla.MLA_ERR_UNSUPPORTED), ("page_size", 32, mla.MLA_ERR_UNSUPPORTED),
+                             ("B", 0, mla.MLA_ERR_INVALID_ARG), ("scale", -1.0, mla.MLA_ERR_INVALID_ARG)]:
+        d = mla.make_dims(2, 1, 16, 4, 8)
+        setattr(d, field, val)
+        with pytest.raises(mla.MlaError) as e:
+            mla.plan(d, [256, 256], 4)
+        assert e.value.code == code, field
+    with pytest.raises(mla.MlaError) as e:
+        mla.plan(good, [256, 257], 4)                 # longer than max_blocks * 64
+    assert e.value.code == mla.MLA_ERR_INVALID_ARG and "seq_lens[1]" in str(e.value)
+    with pytest.raises(mla.MlaError) as e:
+        mla.plan(mla.make_dims(1, 2, 16, 4, 8), [1], 4)   # T < s_q
+    assert e.value.code == mla.MLA_ERR_INVALID_ARG
+    # null / misaligned device pointers are rejected before any CUDA call
+    lib = mla._lib
+    assert lib.mla_absorb_q(None, 16, 16, 4, 16, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_absorb_q(16, 16, 16, 0, 16, None) == mla.MLA_ERR_UNSUPPORTED
+    assert lib.mla_out_uv(16, 24, 16, 4, 16, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode_attn(ctypes.byref(good), 16, 16, 16, 16, 16, 16, 4, None, None, None, None,
+                               None, None) == mla.MLA_ERR_INVALID_ARG
+    assert b"o_lat" in lib.mla_last_error_string()
+    assert lib.mla_combine(ctypes.byref(good), 16, None, None, 16, None, None) == mla.MLA_ERR_INVALID_ARG
+    small = (ctypes.c_int32 * 4)()
+    assert lib.mla_plan(ctypes.byref(good), (ctypes.c_int32 * 2)(256, 256), 4, small, 16,
+                        None) == mla.MLA_ERR_WORKSPACE_TOO_SMALL
