@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of one absorbed-MLA decode step (one layer) on B200.
+
+A step is the whole decode path on one batch: mla_absorb_q -> mla_decode_attn
+-> mla_combine -> mla_out_uv, with inputs resident in HBM.  The default
+workload is the DeepSeek-V2-shaped decode batch (B=32 sequences x 1 query
+token, 128 heads, T=4096 keys each, 64-token pages in a random permutation of
+the pool).  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by its own CUDA
+events on the launching stream, with L2 flushed before every step by writing
+a 256 MB buffer (outside the events); the K-step region is bracketed by a
+barrier and torch.cuda.synchronize() on both sides; ms_per_step is the mean
+per-step event time, max over ranks.  The attention kernel alone is timed the
+same way for the roofline.  `e2e` repeats the step through the public
+Decoder API with the step's inputs (queries, page table) copied from pinned
+host memory and the output copied back, inside the timed region.
+
+Multi-GPU (torchrun, one process per GPU): data-parallel replicas.  Each rank
+decodes its own batch of the same shape (weak scaling); no collective runs on
+the data path; timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode tokens/s and effective cache TB/s (% of B200 roofline)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+DECODE_SOURCES = ("head_latent_attention_04_b200/csrc/decode_attn.cu",
+                  "head_latent_attention_04_b200/csrc/ptx.cuh")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="v2_4k",
+                    choices=["tiny", "v2_4k", "varlen", "long128k", "mtp2"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of a CUDA graph")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- accounting
+def algorithmic(seq_lens, s_q, H, causal=True):
+    """Algorithmic bytes / FLOPs of the step and of the attention kernel.
+
+    Per attended (query, key) pair: 2*h*(2*d_c + d_R) FLOPs (QK over 576 +
+    PV over 512 per head).  Per cached token: 576 bf16 = 1152 B, read once
+    and shared by all heads and all s_q query tokens of its sequence.
+    """
+    T = np.asarray(seq_lens, dtype=np.int64)
+    N = len(T) * s_q
+    pairs = int(sum(int(t) - s_q + 1 + i if causal else int(t) for t in T for i in range(s_q)))
+    cache = int(T.sum()) * 576 * 2
+    w_bytes = 2 * 512 * H * 128 * 2
+    attn_flops = pairs * 2 * H * (2 * 512 + 64)
+    bmm_flops = 2 * (2 * N * H * 128 * 512)
+    q_in = N * H * (128 + 64) * 2
+    out_b = N * H * 128 * 2
+    attn_bytes = cache + N * H * (512 + 64) * 2 + N * H * 512 * 2
+    return dict(N=N, pairs=pairs, cache_bytes=cache, step_bytes=cache + w_bytes + q_in + out_b,
+                step_flops=attn_flops + bmm_flops, attn_bytes=attn_bytes, attn_flops=attn_flops)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config: str):
+    """DRAM bytes per attention launch from a committed ncu summary, if it still
+    describes the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    e = d.get(config)
+    if not e or e.get("source_hash") != decode_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, uuid: str | None, index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            if uuid:
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "samples": len(self.samples), "reasons": names}
+
+
+# ----------------------------------------------------------------------------- CPU oracle sample
+def cpu_oracle_sample(w, seconds: float, max_rows: int | None = None):
+    """Times the float64 oracle on whole query rows (all heads, full context) of
+    the workload until `seconds` of CPU work; returns (rows/s, rows, seconds, cores)."""
+    from oracle import mla_oracle as O
+    cores = len(os.sched_getaffinity(0))
+    w_uk = w.w_uk.cpu().double().numpy()
+    w_uv = w.w_uv.cpu().double().numpy()
+    done, t0 = 0, time.perf_counter()
+    order = list(range(w.B))
+    for b in order:
+        rows = slice(b * w.s_q, (b + 1) * w.s_q)
+        cache = w.cache_rows(b).cpu().double().numpy()
+        O.mla_decode(w.q_nope[rows].cpu().double().numpy(), w.q_rope[rows].cpu().double().numpy(),
+                     [cache], w_uk, w_uv, w.s_q, with_intermediates=False)
+        done += w.s_q
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_rows and done >= max_rows):
+            break
+    el = time.perf_counter() - t0
+    return done / el, done, el, cores
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    from head_latent_attention_04_b200 import workloads as W
+    w = W.preset_workload(args.config, device="cpu")
+    rows_per_step = w.s_q                       # one sequence's query rows per step
+    K, Wm = args.steps, args.warmup
+    per_row_budget = None
+    # warm-up on one row, then time K steps of one sequence each (cycling through the batch)
+    from oracle import mla_oracle as O
+    w_uk = w.w_uk.double().numpy()
+    w_uv = w.w_uv.double().numpy()
+    caches = {}
+
+    def step(i):
+        b = i % w.B
+        rows = slice(b * w.s_q, (b + 1) * w.s_q)
+        if b not in caches:
+            caches[b] = w.cache_rows(b).double().numpy()
+        O.mla_decode(w.q_nope[rows].double().numpy(), w.q_rope[rows].double().numpy(), [caches[b]],
+                     w_uk, w_uv, w.s_q, with_intermediates=False)
+
+    for i in range(min(Wm, 1)):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(K):
+        step(i)
+    el = time.perf_counter() - t0
+    value = K * rows_per_step / el
+    cores = len(os.sched_getaffinity(0))
+    sample = f"{K} steps x {rows_per_step} query row(s) of {args.config}, all {w.n_heads} heads, full context"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": Wm, "ms_per_step": 1e3 * el / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.config, w),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def workload_config(name, w):
+    T = np.asarray(w.seq_lens)
+    return {"workload": name, "B": int(w.B), "s_q": int(w.s_q), "n_heads": int(w.n_heads),
+            "d_c": 512, "d_rope": 64, "d_nope": 128, "d_v": 128, "page_size": 64,
+            "T_total": int(T.sum()), "T_min": int(T.min()), "T_max": int(T.max()),
+            "pool": w.meta.get("pool"), "seed": w.meta.get("seed"),
+            "l2": "flushed before every step (256 MB write, outside the step events)"}
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    from head_latent_attention_04_b200 import mla
+    from head_latent_attention_04_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    preset = W.PRESETS[args.config]
+    w = W.preset_workload(args.config, device=dev, seed=preset.seed + 1000 * rank)
+    acc = algorithmic(w.seq_lens, w.s_q, w.n_heads)
+    bt = torch.as_tensor(w.block_table, device=dev)
+    dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dec.run(w.q_nope, w.q_rope, w.kv_pool, bt, w.w_uk, w.w_uv)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if dec.status.item() != 0:
+        raise RuntimeError(f"device status {dec.status.item():#x} after warm-up")
+
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+        except Exception as e:  # fall back to eager launches
+            print(f"[bench] CUDA graph capture failed ({e}); eager launches", file=sys.stderr)
+            graph = None
+    run_step = graph.replay if graph is not None else step
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid, local_rank)
+    barrier()
+    t_wall = time.perf_counter()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            run_step()
+            ev[i][1].record(stream)
+        # the attention kernel alone, same hygiene, for the roofline
+        for i in range(K):
+            flush.zero_()
+            ea[i][0].record(stream)
+            mla.decode_attn(dec.dims, dec.q_lat, w.q_rope, w.kv_pool, bt, dec.seq_lens_dev, dec.plan_dev,
+                            dec.num_clusters, dec.o_part, dec.lse_part, dec.o_lat, dec.lse, dec.status)
+            ea[i][1].record(stream)
+        barrier()
+    t_wall = time.perf_counter() - t_wall
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    attn_ms = [a.elapsed_time(b) for a, b in ea]
+    ms_local = statistics.fmean(step_ms)
+    attn_local = statistics.fmean(attn_ms)
+
+    # e2e: the public API with host buffers (queries + page table in, output out)
+    qn_h = w.q_nope.cpu().pin_memory()
+    qr_h = w.q_rope.cpu().pin_memory()
+    bt_h = torch.as_tensor(w.block_table).pin_memory()
+    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    qn_d, qr_d, bt_d = torch.empty_like(w.q_nope), torch.empty_like(w.q_rope), torch.empty_like(bt)
+    h2d = qn_h.numel() * 2 + qr_h.numel() * 2 + bt_h.numel() * 4
+    d2h = out_h.numel() * 2
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier()
+    for i in range(K):
+        flush.zero_()
+        ee[i][0].record(stream)
+        qn_d.copy_(qn_h, non_blocking=True)
+        qr_d.copy_(qr_h, non_blocking=True)
+        bt_d.copy_(bt_h, non_blocking=True)
+        r = dec.run(qn_d, qr_d, w.kv_pool, bt_d, w.w_uk, w.w_uv)
+        out_h.copy_(r.out, non_blocking=True)
+        ee[i][1].record(stream)
+    barrier()
+    e2e_local = statistics.fmean(a.elapsed_time(b) for a, b in ee)
+    status = int(dec.status.item())
+
+    if world > 1:
+        t = torch.tensor([ms_local, attn_local, e2e_local], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, attn, e2e = t.tolist()
+        st = torch.tensor([status], dtype=torch.int32, device=dev)
+        torch.distributed.all_reduce(st, op=torch.distributed.ReduceOp.MAX)
+        status = int(st.item())
+    else:
+        ms, attn, e2e = ms_local, attn_local, e2e_local
+    if graph is not None:
+        del graph
+    if rank != 0:
+        return None
+
+    peaks, peak_src = load_peaks()
+    tensor_bound = acc["attn_flops"] / (peaks["bf16_tflops"] * 1e12) > acc["attn_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        achieved = acc["attn_flops"] / (attn * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        achieved = acc["attn_bytes"] / (attn * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof.update({"traffic": recorded_traffic(args.config), "kernel": "mla_decode_kernel",
+                 "alg_bytes_per_launch": acc["attn_bytes"], "alg_flops_per_launch": acc["attn_flops"],
+                 "kernel_ms": attn, "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'}, burst)"})
+    step_roof_s = max(acc["step_bytes"] / (peaks["hbm_gbs"] * 1e9), acc["step_flops"] / (peaks["bf16_tflops"] * 1e12))
+    tokens = acc["N"] * world
+    res = {
+        "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(args.config, w), parallelism=f"dp{world} (independent replicas)",
+                       num_clusters=dec.num_clusters, split_slots=dec.num_slots,
+                       graph=graph is not None),
+        "cache_tbs": acc["cache_bytes"] * world / (ms * 1e-3) / 1e12,
+        "attn_cache_tbs": acc["cache_bytes"] / (attn * 1e-3) / 1e12,
+        "tflops": acc["step_flops"] * world / (ms * 1e-3) / 1e12,
+        "step_roofline_frac": step_roof_s / (ms * 1e-3),
+        "roofline": roof,
+        "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+        "gpu_launches": K * dec.launches_per_step + K,
+        "clocks": sampler.summary(),
+        "device_status": status,
+        "wall_s_timed_region": t_wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, rows, secs, cores = cpu_oracle_sample(w, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "sample": f"{rows} query rows of {args.config} (all heads, full context), "
+                                         f"{secs:.1f} s, float64 order-1 oracle"}
+    return res
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        import torch
+        if world > 1:
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local_rank))
+        try:
+            res = run_ours(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

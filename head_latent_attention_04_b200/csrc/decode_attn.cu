@@ -442,6 +442,13 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   cluster_sync();   // no CTA leaves while its peer may still write into its shared memory
 }
 
+// Set once per process, so that later launches can be captured in a CUDA graph.
+cudaError_t decode_smem_attr() {
+  static cudaError_t e =
+      cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  return e;
+}
+
 }  // namespace
 
 mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
@@ -485,7 +492,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
   p.num_clusters = num_clusters;
   p.scale_log2 = d.scale * 1.4426950408889634f;
 
-  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = decode_smem_attr();
   if (e == cudaSuccess) {
     mla_decode_kernel<<<2 * num_clusters, 192, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tm_kv, tm_rope, tm_q, p);
     e = cudaGetLastError();
@@ -495,7 +502,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
 }
 
 mla_status_t decode_max_clusters(int32_t* n) {
-  cudaError_t e = cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaError_t e = decode_smem_attr();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "max clusters: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);

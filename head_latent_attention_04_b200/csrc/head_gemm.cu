@@ -172,18 +172,18 @@ mla_status_t launch_head_gemm(bool a_mn, const void* weight, const void* act, vo
   dim3 grid(m_total / kBM, n_heads, (n_tokens + bn - 1) / bn);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (a_mn) {
-    e = cudaFuncSetAttribute(head_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) {
+  // Attributes are set once per process (outside any later stream capture).
+  static cudaError_t attr_mn = cudaFuncSetAttribute(
+      head_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  static cudaError_t attr_k = cudaFuncSetAttribute(
+      head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  e = a_mn ? attr_mn : attr_k;
+  if (e == cudaSuccess) {
+    if (a_mn)
       head_gemm_kernel<true><<<grid, 128, kSmemBytes, s>>>(tA, tB, p);
-      e = cudaGetLastError();
-    }
-  } else {
-    e = cudaFuncSetAttribute(head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e == cudaSuccess) {
+    else
       head_gemm_kernel<false><<<grid, 128, kSmemBytes, s>>>(tA, tB, p);
-      e = cudaGetLastError();
-    }
+    e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "head_gemm launch: %s", cudaGetErrorString(e));
   return MLA_OK;
