@@ -355,8 +355,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         status = int(st.item())
     else:
         ms, attn, e2e = ms_local, attn_local, e2e_local
-    if graph is not None:
-        del graph
+    used_graph = graph is not None
+    del graph
     if rank != 0:
         return None
 
@@ -381,7 +381,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(args.config, w), parallelism=f"dp{world} (independent replicas)",
                        num_clusters=dec.num_clusters, split_slots=dec.num_slots,
-                       graph=graph is not None),
+                       graph=used_graph),
         "cache_tbs": acc["cache_bytes"] * world / (ms * 1e-3) / 1e12,
         "attn_cache_tbs": acc["cache_bytes"] / (attn * 1e-3) / 1e12,
         "tflops": acc["step_flops"] * world / (ms * 1e-3) / 1e12,

@@ -45,22 +45,29 @@ using namespace ptx;
 
 constexpr int kPage = 64;
 constexpr int kRows = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kChunkBytes = kPage * 128;                     // 64 keys x 64 latent cols (SW128)
 constexpr int kRopeBytes = kPage * 64;                       // 64 keys x 32 rope cols (SW64)
 constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;    // 36 KB: half a page
 constexpr int kQRopeBytes = kRows * 64;                      // 128 rows x 32 rope cols (SW64)
 constexpr int kPBytes = kRows * 128;                         // 128 rows x 64 keys bf16 (SW128)
-constexpr int kXRow = 64 * 4 + 16;                           // padded fp32 score row
-constexpr int kXBytes = kRows * kXRow;
+constexpr int kXRow = 64 * 2;                                // fp16 score row, 16B chunks XOR (row & 7)
+constexpr int kXBytes = kRows * kXRow;                       // one exchange tile (16 KB)
 
 constexpr int kOffKV = 0;
 constexpr int kOffQRope = kOffKV + kStages * kStageBytes;
 constexpr int kOffP = kOffQRope + kQRopeBytes;
 constexpr int kOffX = kOffP + 2 * kPBytes;
-constexpr int kOffBar = kOffX + kXBytes;
-constexpr int kNumBars = 2 * kStages + 16;
+constexpr int kOffXS = kOffX + 2 * kXBytes;            // send staging, 2 tiles
+constexpr int kOffPMax = kOffXS + 2 * kXBytes;         // fp32 [2 pages][2 halves][128] half-row maxima
+constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;      // fp32 [2 items][2 halves][128] half-row sums
+constexpr int kOffBar = kOffLSum + 4 * kRows * 4;
+constexpr int kNumBars = 2 * kStages + 34;
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+
+constexpr int kThreads = 448;            // 14 warps: TMA, MMA, 4 exchange, 8 softmax
+constexpr int kXchgWarp0 = 2, kSoftWarp0 = 6;
+constexpr int kSoftWarps = 8;
 
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384, kTmemCols = 512;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -84,7 +91,13 @@ struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full, q_empty;
   uint64_t s_full[2], s_free[2], p_full[2], p_free[2];
-  uint64_t o_full, o_free, x_full, x_free, mma_done, pad;
+  uint64_t x_recv[2];    // peer's fp16 partial scores landed in x buffer b (1 arrival + 16 KB tx)
+  uint64_t x_sendok[2];  // peer has consumed its x buffer b, which this CTA may refill (8 remote arrivals)
+  uint64_t o_full, o_free, mma_done, pad;
+  uint64_t pmax[2][4];   // the two softmax warps of row quarter q posted their page-b half-row maxima
+  uint64_t lsum[4];      // the two softmax warps of row quarter q posted their half-row sums (per item)
+  uint64_t stg_ok[2];    // send staging tile b may be rewritten (issuer, after the old copy read it)
+  uint64_t stg_full[2];  // send staging tile b written by the 4 sender warps
 };
 static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
 
@@ -99,7 +112,13 @@ __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity
   return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort));
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rope,
                   const __grid_constant__ CUtensorMap tm_qrope, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -108,6 +127,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   uint8_t* s_qrope = smem + kOffQRope;
   uint8_t* s_p = smem + kOffP;
   uint8_t* s_x = smem + kOffX;
+  uint8_t* s_xs = smem + kOffXS;
+  float* s_pmax = reinterpret_cast<float*>(smem + kOffPMax);
+  float* s_lsum = reinterpret_cast<float*>(smem + kOffLSum);
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + sizeof(Bars));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -130,19 +152,29 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->q_full, 1 + kRows);
+    mbar_init(&bars->q_full, 1 + kSoftWarps);
     mbar_init(&bars->q_empty, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], kRows);
-      mbar_init(&bars->p_full[b], kRows);
+      mbar_init(&bars->s_free[b], 4 + kSoftWarps);
+      mbar_init(&bars->p_full[b], kSoftWarps);
       mbar_init(&bars->p_free[b], 1);
+      mbar_init(&bars->x_recv[b], 1);
+      mbar_init(&bars->x_sendok[b], kSoftWarps);
     }
+    for (int b = 0; b < 2; ++b) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);   // armed for pages 0, 1
     mbar_init(&bars->o_full, 1);
-    mbar_init(&bars->o_free, kRows);
-    mbar_init(&bars->x_full, kRows);
-    mbar_init(&bars->x_free, kRows);
+    mbar_init(&bars->o_free, kSoftWarps);
     mbar_init(&bars->mma_done, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bars->pmax[0][q], 2);
+      mbar_init(&bars->pmax[1][q], 2);
+      mbar_init(&bars->lsum[q], 2);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->stg_ok[b], 1);
+      mbar_init(&bars->stg_full[b], 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_kv);
@@ -258,135 +290,211 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mma_commit(&bars->mma_done);
       mbar_wait(&bars->mma_done, 0, nullptr);   // no MMA may still write TMEM at dealloc
     }
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue
-    const int quarter = warp & 3;                 // TMEM lanes this warp may touch
-    const int r = quarter * 32 + lane;            // head row = TMEM lane
+  } else if (warp < kSoftWarp0) {
+    // ------------------------------------------------------------ score sender (4 warps)
+    // This CTA's partial scores (its 288 columns), rounded to fp16, go to the
+    // peer's exchange tile b by one bulk copy that completes on the peer's
+    // x_recv[b].  Thread = one row (TMEM lane), 64 keys; the tile is staged
+    // locally with 16-byte chunks XOR-swizzled by (row & 7).
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t x_row = smem_u32(s_x) + r * kXRow;
-    const uint32_t x_row_peer = mapa(x_row, peer);
-    const uint32_t x_full_peer = mapa(smem_u32(&bars->x_full), peer);
-    const uint32_t x_free_peer = mapa(smem_u32(&bars->x_free), peer);
-    const float* xr = reinterpret_cast<const float*>(s_x + r * kXRow);
-    uint8_t* prow0 = s_p + r * 128;
+    const bool issuer = (warp == 2 && lane == 0);
+    const uint32_t x_peer = mapa(smem_u32(s_x), peer);
+    const uint32_t x_recv_peer = mapa(smem_u32(&bars->x_recv[0]), peer);
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
-      const int row = w[kItRow], pb = w[kItPageBegin], n = w[kItPageEnd] - pb;
-      const int kv_len = w[kItKvLen], slot = w[kItSlot];
+      const int n = w[kItPageEnd] - w[kItPageBegin];
+      for (int j = 0; j < n; ++j) {
+        const int gj = g + j, b = gj & 1;
+        uint32_t v[64];
+        if (!warp_wait(&bars->s_full[b], (gj >> 1) & 1, abort_flag)) goto xchg_fail;
+        tc_fence_after();
+        tmem_ld32(tmem + lane_addr + kTmemS + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tmem + lane_addr + kTmemS + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[b]);
+        uint32_t hv[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) hv[k] = pack_f16(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+        // staging tile b is reusable once the copy issued two pages ago has read it
+        if (issuer) {
+          bulk_wait_read<1>();
+          mbar_arrive(&bars->stg_ok[b]);
+        }
+        if (!warp_wait(&bars->stg_ok[b], (gj >> 1) & 1, abort_flag)) goto xchg_fail;
+        {
+          uint8_t* row = s_xs + b * kXBytes + r * kXRow;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4*>(row + ((k ^ (r & 7)) << 4)) =
+                make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->stg_full[b]);
+        if (issuer) {
+          if (!mbar_wait(&bars->stg_full[b], (gj >> 1) & 1, abort_flag)) goto xchg_fail;
+          if (gj >= 2 && !mbar_wait(&bars->x_sendok[b], ((gj >> 1) - 1) & 1, abort_flag)) goto xchg_fail;
+          bulk_copy_to_peer(x_peer + b * kXBytes, smem_u32(s_xs + b * kXBytes), kXBytes, x_recv_peer + 8 * b);
+          bulk_commit();
+        }
+      }
+      g += n;
+    }
+    goto xchg_done;
+  xchg_fail:
+    *abort_flag = 1;
+    if (lane == 0) report(p.status, MLA_STATUS_TIMEOUT);
+  xchg_done:
+    if (issuer) bulk_wait_read<0>();   // the staging tiles must outlive their copies
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue (8 warps)
+    // Thread = (row r, key half c): keys [32c, 32c+32) of each page, output
+    // columns [128c, 128c+128) of this CTA's 256.
+    const int quarter = warp & 3;
+    const int c = (warp - kSoftWarp0) >> 2;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    uint8_t* prow0 = s_p + r * 128;
+    const float sl2 = p.scale_log2;
+    const uint32_t x_sendok_peer = mapa(smem_u32(&bars->x_sendok[0]), peer);
+    int g = 0;
+    for (int it = it_begin; it < it_end; ++it) {
+      const int32_t* w = items + (size_t)it * kItemWords;
+      const int row = w[kItRow], pb = w[kItPageBegin], n = w[kItPageEnd] - pb, slot = w[kItSlot];
+      const int kv_len = w[kItKvLen];
       const int ii = it - it_begin;
 
-      // q_lat half of this row -> TMEM (bf16 pairs, A operand of the QK product)
+      // this thread's 128 q_lat columns -> TMEM (bf16 pairs, A operand of the QK product)
       if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto softmax_fail;
       {
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)row * p.n_heads + r) * 512 + 256 * rank);
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)row * p.n_heads + r) * 512 +
+                                                          256 * rank + 128 * c);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int h = 0; h < 2; ++h) {
           uint32_t v[32];
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            uint4 q = r < p.n_heads ? __ldg(src + c * 8 + k) : make_uint4(0, 0, 0, 0);
+            const uint4 q = r < p.n_heads ? __ldg(src + h * 8 + k) : make_uint4(0, 0, 0, 0);
             v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
           }
-          tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+          tmem_st32(tmem + lane_addr + kTmemQ + 64 * c + 32 * h, v);
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars->q_full);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_full);
       }
 
       float m_ref = -CUDART_INF_F, l_run = 0.f;
       for (int j = 0; j < n; ++j) {
         const int gj = g + j, b = gj & 1;
-        float sc[64];
-        // own partial scores
+        // full score = fp16(own partial) + fp16(peer partial), identical in both CTAs
+        if (!warp_wait(&bars->x_recv[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
         if (!warp_wait(&bars->s_full[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
         tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + kTmemS + 64 * b + 32 * c, v);
+        uint4 pr[4];
         {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_addr + kTmemS + 64 * b, v);
-          tmem_ld_wait();
+          const uint8_t* xrow = s_x + b * kXBytes + r * kXRow;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) sc[k] = __uint_as_float(v[k]);
-          tmem_ld32(tmem + lane_addr + kTmemS + 64 * b + 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) sc[32 + k] = __uint_as_float(v[k]);
+          for (int k = 0; k < 4; ++k)
+            pr[k] = *reinterpret_cast<const uint4*>(xrow + (((4 * c + k) ^ (r & 7)) << 4));
         }
+        tmem_ld_wait();
         tc_fence_before();
-        mbar_arrive(&bars->s_free[b]);
-
-        // exchange partial scores with the peer CTA through distributed shared memory
-        if (gj >= 1 && !warp_wait_cluster(&bars->x_free, (gj - 1) & 1, abort_flag)) goto softmax_fail;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free[b]);
+        uint32_t used = 0;
+        {
+          const uint32_t* pw = reinterpret_cast<const uint32_t*>(pr);
 #pragma unroll
-        for (int k = 0; k < 16; ++k)
-          st_cluster_v4(x_row_peer + 16 * k, sc[4 * k], sc[4 * k + 1], sc[4 * k + 2], sc[4 * k + 3]);
-        mbar_arrive_cluster(x_full_peer);
-        if (!warp_wait_cluster(&bars->x_full, gj & 1, abort_flag)) goto softmax_fail;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float4 o = *reinterpret_cast<const float4*>(xr + 4 * k);
-          sc[4 * k] += o.x; sc[4 * k + 1] += o.y; sc[4 * k + 2] += o.z; sc[4 * k + 3] += o.w;
+          for (int k = 0; k < 16; ++k) {
+            const float2 own = round_f16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+            const float2 oth = unpack_f16x2(pw[k]);
+            used |= pw[k];
+            v[2 * k] = __float_as_uint(own.x + oth.x);
+            v[2 * k + 1] = __float_as_uint(own.y + oth.y);
+          }
         }
-        mbar_arrive_cluster(x_free_peer);
-
-        // scale (log2 domain), mask keys past kv_len, running max with lazy reference
-        const int tok0 = (pb + j) * kPage;
-        float mx = -CUDART_INF_F;
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          sc[k] = (tok0 + k < kv_len) ? sc[k] * p.scale_log2 : -CUDART_INF_F;
-          mx = fmaxf(mx, sc[k]);
+        // exchange tile b is consumed: re-arm it for page gj + 2, then let the peer refill it
+        {
+          uint32_t ok_addr = x_sendok_peer + 8 * b;
+          asm volatile("" : "+r"(ok_addr) : "r"(used));   // issue only after the tile was read
+          __syncwarp();
+          if (lane == 0) {
+            if (warp == kSoftWarp0) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);
+            mbar_arrive_relaxed_cluster(ok_addr);
+          }
         }
+        const int tok0 = (pb + j) * kPage + 32 * c;
+        if (tok0 + 32 > kv_len) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (tok0 + k >= kv_len) v[k] = __float_as_uint(-CUDART_INF_F);
+        }
+        float mloc = __uint_as_float(v[0]);
+#pragma unroll
+        for (int k = 1; k < 32; ++k) mloc = fmaxf(mloc, __uint_as_float(v[k]));
+        s_pmax[(b * 2 + c) * kRows + r] = mloc;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->pmax[b][quarter]);
+        if (!warp_wait(&bars->pmax[b][quarter], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
+        const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kRows + r]) * sl2;
+
+        // lazy reference max (log2 domain): move it only when the row max grows by > 2^8
         const float m_new = fmaxf(m_ref, mx);
         const bool move = (m_ref == -CUDART_INF_F) ? (m_new != -CUDART_INF_F)
                                                    : (m_new > m_ref + kRescaleThreshold);
         float alpha = 1.f;
         if (move) {
-          alpha = (m_ref == -CUDART_INF_F) ? 0.f : exp2f(m_ref - m_new);
+          alpha = (m_ref == -CUDART_INF_F) ? 0.f : ex2(m_ref - m_new);
           m_ref = m_new;
         }
-        const float base = (m_ref == -CUDART_INF_F) ? 0.f : m_ref;
-        uint32_t pk[32];
-        float psum = 0.f;
+        const float nb = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+        uint32_t pk[16];
+        float ps = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float e0 = exp2f(sc[2 * k] - base), e1 = exp2f(sc[2 * k + 1] - base);
+        for (int k = 0; k < 16; ++k) {
+          const float e0 = ex2(fmaf(__uint_as_float(v[2 * k]), sl2, nb));
+          const float e1 = ex2(fmaf(__uint_as_float(v[2 * k + 1]), sl2, nb));
           pk[k] = pack_bf16(e0, e1);
-          const __nv_bfloat162 rb = *reinterpret_cast<__nv_bfloat162*>(&pk[k]);
-          psum += __bfloat162float(rb.x) + __bfloat162float(rb.y);
+          ps += e0 + e1;
         }
-        l_run = l_run * alpha + psum;
+        l_run = l_run * alpha + ps;
 
-        // P buffer b is free once the PV product two pages back has completed
         if (gj >= 2 && !warp_wait(&bars->p_free[b], ((gj >> 1) - 1) & 1, abort_flag)) goto softmax_fail;
-        // rescale O in TMEM when this row's reference max moved (rare after the first page)
         if (__any_sync(0xffffffffu, move && j > 0)) {
           if (!warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
           tc_fence_after();
           const float a = (move && j > 0) ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_addr + kTmemO + 32 * c, v);
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_addr + kTmemO + 128 * c + 32 * q, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * a);
-            tmem_st32(tmem + lane_addr + kTmemO + 32 * c, v);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+            tmem_st32(tmem + lane_addr + kTmemO + 128 * c + 32 * q, o);
           }
           tmem_st_wait();
         }
-        // P row (64 keys, bf16) into the 128B-swizzled K-major A tile
         {
           uint8_t* prow = prow0 + b * kPBytes;
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(prow + ((k ^ (r & 7)) << 4)) =
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(prow + (((4 * c + k) ^ (r & 7)) << 4)) =
                 make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&bars->p_full[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->p_full[b]);
       }
 
       // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot
@@ -394,38 +502,45 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         const int gl = g + n - 1;
         if (!warp_wait(&bars->o_full, gl & 1, abort_flag)) goto softmax_fail;
         tc_fence_after();
+        float* ls = s_lsum + (ii & 1) * 2 * kRows;    // [item parity][half][row]
+        ls[c * kRows + r] = l_run;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->lsum[quarter]);
+        if (!warp_wait(&bars->lsum[quarter], ii & 1, abort_flag)) goto softmax_fail;
+        l_run = ls[r] + ls[kRows + r];             // same order in both halves
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const bool valid = r < p.n_heads;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_addr + kTmemO + 32 * c, v);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_addr + kTmemO + 128 * c + 32 * q, o);
           tmem_ld_wait();
           if (!valid) continue;
-          const int col = 256 * rank + 32 * c;
+          const int col = 256 * rank + 128 * c + 32 * q;
           if (slot < 0) {
             uint4* dst = reinterpret_cast<uint4*>(p.o_lat + ((size_t)row * p.n_heads + r) * 512 + col);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(pack_bf16(__uint_as_float(v[8 * k]) * inv_l, __uint_as_float(v[8 * k + 1]) * inv_l),
-                                  pack_bf16(__uint_as_float(v[8 * k + 2]) * inv_l, __uint_as_float(v[8 * k + 3]) * inv_l),
-                                  pack_bf16(__uint_as_float(v[8 * k + 4]) * inv_l, __uint_as_float(v[8 * k + 5]) * inv_l),
-                                  pack_bf16(__uint_as_float(v[8 * k + 6]) * inv_l, __uint_as_float(v[8 * k + 7]) * inv_l));
+              dst[k] = make_uint4(pack_bf16(__uint_as_float(o[8 * k]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
+                                  pack_bf16(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
+                                  pack_bf16(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
+                                  pack_bf16(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
           } else {
             float4* dst = reinterpret_cast<float4*>(p.o_part + ((size_t)slot * p.n_heads + r) * 512 + col);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              dst[k] = make_float4(__uint_as_float(v[4 * k]) * inv_l, __uint_as_float(v[4 * k + 1]) * inv_l,
-                                   __uint_as_float(v[4 * k + 2]) * inv_l, __uint_as_float(v[4 * k + 3]) * inv_l);
+              dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                   __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
           }
         }
-        if (valid && rank == 0) {
+        if (valid && rank == 0 && c == 0) {
           const float lse = (l_run > 0.f) ? (m_ref + __log2f(l_run)) * kLn2 : -CUDART_INF_F;
           if (slot >= 0) p.lse_part[(size_t)slot * p.n_heads + r] = lse;
           else if (p.lse_out) p.lse_out[(size_t)row * p.n_heads + r] = lse;
         }
         tc_fence_before();
-        mbar_arrive(&bars->o_free);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->o_free);
       }
       g += n;
     }
@@ -438,7 +553,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  __syncwarp();
   cluster_sync();   // no CTA leaves while its peer may still write into its shared memory
 }
 
@@ -494,7 +611,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
 
   cudaError_t e = decode_smem_attr();
   if (e == cudaSuccess) {
-    mla_decode_kernel<<<2 * num_clusters, 192, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tm_kv, tm_rope, tm_q, p);
+    mla_decode_kernel<<<2 * num_clusters, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tm_kv, tm_rope, tm_q, p);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
@@ -506,7 +623,7 @@ mla_status_t decode_max_clusters(int32_t* n) {
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "max clusters: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

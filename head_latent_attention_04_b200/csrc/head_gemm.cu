@@ -10,9 +10,11 @@
 // CTA).  Reading W_UK / W_UV (16.8 MB each at 128 heads) dominates, as the
 // izhida.com answer notes for the W_V product of a batched GEMV.
 //
-// One CTA per (128-row M tile, head, token tile).  Warp 0 streams 64-wide K
-// slices through a 4-stage TMA ring, warp 1 issues tcgen05.mma into a TMEM
-// accumulator of 128 lanes x BN columns, and all four warps drain it.
+// One CTA per (head, token tile), covering all M tiles of that head (4 for
+// W_UK, 1 for W_UV), so a 128-head batch runs as a single wave.  Warp 0
+// streams (M tile, 64-wide K slice) pairs through a 4-stage TMA ring, warp 1
+// issues tcgen05.mma into one TMEM accumulator of 128 lanes x BN columns per
+// M tile, and all four warps drain them.
 #include "mla_internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -30,7 +32,6 @@ constexpr int kStages = 4;
 constexpr int kMaxBN = 128;
 constexpr int kABytes = kBM * kBK * 2;       // 16 KB
 constexpr int kBBytesMax = kMaxBN * kBK * 2; // 16 KB
-constexpr int kTmemCols = 128;
 constexpr int kSmemBytes = kStages * (kABytes + kBBytesMax) + 1024 /*align*/ + 256 /*barriers*/;
 
 struct Params {
@@ -58,8 +59,11 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int m0 = blockIdx.x * kBM, h = blockIdx.y, n0 = blockIdx.z * p.bn;
-  const int k_steps = p.k_total / kBK;
+  const int h = blockIdx.y, n0 = blockIdx.z * p.bn;
+  const int k_chunks = p.k_total / kBK;
+  const int m_tiles = p.m_total / kBM;
+  const int k_steps = m_tiles * k_chunks;            // (m tile, k chunk) pairs, m-major
+  const uint32_t tmem_cols = m_tiles == 1 ? 128u : 512u;
   const uint32_t b_bytes = p.bn * kBK * 2;
 
   if (threadIdx.x == 0) {
@@ -74,7 +78,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -84,9 +88,9 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
   if (warp == 0 && lane == 0) {
     // producer
-    for (int kc = 0; kc < k_steps; ++kc) {
-      const int s = kc % kStages;
-      if (kc >= kStages && !mbar_wait(&empty[s], ((kc / kStages) - 1) & 1, abort_flag)) {
+    for (int ks = 0; ks < k_steps; ++ks) {
+      const int s = ks % kStages, mt = ks / k_chunks, kc = ks % k_chunks;
+      if (ks >= kStages && !mbar_wait(&empty[s], ((ks / kStages) - 1) & 1, abort_flag)) {
         *abort_flag = 1;
         break;
       }
@@ -97,16 +101,16 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tma_load_3d(sA + s * kABytes + kABytes / 2, &tmA, &full[s], 64, h, kc * kBK);
       } else {
         // W_UK slice: 128 latent rows of 64 d each
-        tma_load_3d(sA + s * kABytes, &tmA, &full[s], kc * kBK, h, m0);
+        tma_load_3d(sA + s * kABytes, &tmA, &full[s], kc * kBK, h, mt * kBM);
       }
       tma_load_3d(sB + s * kBBytesMax, &tmB, &full[s], kc * kBK, h, n0);
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer
     const uint32_t idesc = idesc_bf16(kBM, p.bn, kAMn ? 1 : 0, 0);
-    for (int kc = 0; kc < k_steps; ++kc) {
-      const int s = kc % kStages;
-      if (!mbar_wait(&full[s], (kc / kStages) & 1, abort_flag)) {
+    for (int ks = 0; ks < k_steps; ++ks) {
+      const int s = ks % kStages, mt = ks / k_chunks, kc = ks % k_chunks;
+      if (!mbar_wait(&full[s], (ks / kStages) & 1, abort_flag)) {
         *abort_flag = 1;
         break;
       }
@@ -117,7 +121,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const uint64_t ad = kAMn ? sdesc(a0 + kk * 2048, kABytes / 2, 1024, kSwizzle128B)
                                  : sdesc(a0 + kk * 32, 16, 1024, kSwizzle128B);
         const uint64_t bd = sdesc(b0 + kk * 32, 16, 1024, kSwizzle128B);
-        mma_ss(tmem, ad, bd, idesc, (kc | kk) != 0);
+        mma_ss(tmem + mt * 128, ad, bd, idesc, (kc | kk) != 0);
       }
       mma_commit(&empty[s]);
     }
@@ -125,28 +129,31 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   }
   __syncwarp();
 
-  // epilogue: thread = accumulator lane = output row m0 + 32*warp + lane
+  // epilogue: thread = accumulator lane = output row mt*128 + 32*warp + lane
   const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0, abort_flag));
   tc_fence_after();
   if (ok) {
-    const int m = m0 + warp * 32 + lane;
     const size_t row_stride = (size_t)p.n_heads * p.m_total;
-    for (int c = 0; c < p.bn; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-      tmem_ld_wait();
+    for (int mt = 0; mt < m_tiles; ++mt) {
+      const int m = mt * kBM + warp * 32 + lane;
+      for (int c = 0; c < p.bn; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * 128 + c, r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int n = n0 + c + j;
-        if (c + j < p.bn && n < p.n_tokens)
-          p.out[(size_t)n * row_stride + (size_t)h * p.m_total + m] =
-              __float2bfloat16_rn(__uint_as_float(r[j]));
+        for (int j = 0; j < 32; ++j) {
+          const int n = n0 + c + j;
+          if (c + j < p.bn && n < p.n_tokens)
+            p.out[(size_t)n * row_stride + (size_t)h * p.m_total + m] =
+                __float2bfloat16_rn(__uint_as_float(r[j]));
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  __syncwarp();
+  if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 }
 
 mla_status_t launch_head_gemm(bool a_mn, const void* weight, const void* act, void* out,
@@ -169,7 +176,7 @@ mla_status_t launch_head_gemm(bool a_mn, const void* weight, const void* act, vo
   if (st != MLA_OK) return st;
 
   Params p{static_cast<__nv_bfloat16*>(out), n_tokens, n_heads, m_total, k_total, bn};
-  dim3 grid(m_total / kBM, n_heads, (n_tokens + bn - 1) / bn);
+  dim3 grid(1, n_heads, (n_tokens + bn - 1) / bn);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   // Attributes are set once per process (outside any later stream capture).
