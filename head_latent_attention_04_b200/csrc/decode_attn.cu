@@ -15,21 +15,25 @@
 // exactly one SM's 512 TMEM columns, leaving no room for S.  So a cluster of
 // two CTAs splits the latent dimension: CTA r owns latent columns
 // [256r, 256r + 256) and RoPE columns [32r, 32r + 32).  Each CTA stages only
-// its half of every cache row (each byte is read from HBM once), computes a
-// partial score over its 288 columns, and the two partial scores are
-// exchanged through distributed shared memory and summed (fp32 addition is
-// commutative, so both CTAs hold bit-identical scores and take identical
-// softmax decisions).  Each CTA then accumulates its 256 output columns.
+// its half of every cache row (each byte is read from HBM once) and computes
+// a partial score over its 288 columns.  The partial scores are rounded to
+// fp16 and exchanged through distributed shared memory (one bulk copy per page,
+// counted on the receiver's mbarrier); both CTAs then form fp16(S0) + fp16(S1) in fp32,
+// which is bit-identical in the pair, so both take the same softmax
+// decisions.  Each CTA accumulates its 256 output columns.
 //
-// TMEM (512 columns): O [0,256) fp32, S double buffer [256,384) fp32,
-// q_lat half [384,512) as the bf16 A operand of the QK product.
+// TMEM (512 columns): O [0,256) fp32, S [256,320) fp32 (released as soon as
+// the sender has read it), P [320,384) as two bf16 buffers (A operand of the
+// PV product), q_lat half [384,512) as bf16 pairs (A operand of QK).
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = MMA issuer and
-// TMEM owner, warps 2-5 = softmax / correction / epilogue (thread = one head
-// row, i.e. one TMEM lane).  The grid is persistent: one cluster per SM pair,
-// each walking the contiguous list of (row, page range) items the host plan
-// gives it.  Every wait is bounded (ptx::kWaitLimitNs); on expiry the CTA sets
-// MLA_STATUS_TIMEOUT and unwinds without trapping.
+// Warp roles (448 threads): warp 0 TMA producer; warp 1 MMA issuer and TMEM
+// owner (one thread, polling the QK and PV streams so neither blocks the
+// other); warps 2-5 score sender (one thread per row, 64 keys); warps 6-13
+// softmax / correction / epilogue (two warps per TMEM lane quarter, one per
+// 32-key half).  The grid
+// is persistent: one cluster per SM pair, each walking the (row, page range)
+// items the host plan gives it.  Every wait is bounded (ptx::kWaitLimitNs);
+// on expiry the CTA sets MLA_STATUS_TIMEOUT and unwinds without trapping.
 #include "mla_internal.h"
 #include "plan_format.h"
 #include "ptx.cuh"
@@ -45,31 +49,27 @@ using namespace ptx;
 
 constexpr int kPage = 64;
 constexpr int kRows = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kChunkBytes = kPage * 128;                     // 64 keys x 64 latent cols (SW128)
 constexpr int kRopeBytes = kPage * 64;                       // 64 keys x 32 rope cols (SW64)
 constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;    // 36 KB: half a page
 constexpr int kQRopeBytes = kRows * 64;                      // 128 rows x 32 rope cols (SW64)
-constexpr int kPBytes = kRows * 128;                         // 128 rows x 64 keys bf16 (SW128)
 constexpr int kXRow = 64 * 2;                                // fp16 score row, 16B chunks XOR (row & 7)
-constexpr int kXBytes = kRows * kXRow;                       // one exchange tile (16 KB)
+constexpr int kXBytes = kRows * kXRow;                       // one score tile (16 KB)
 
 constexpr int kOffKV = 0;
 constexpr int kOffQRope = kOffKV + kStages * kStageBytes;
-constexpr int kOffP = kOffQRope + kQRopeBytes;
-constexpr int kOffX = kOffP + 2 * kPBytes;
-constexpr int kOffXS = kOffX + 2 * kXBytes;            // send staging, 2 tiles
-constexpr int kOffPMax = kOffXS + 2 * kXBytes;         // fp32 [2 pages][2 halves][128] half-row maxima
+constexpr int kOffXPeer = kOffQRope + kQRopeBytes;      // peer's partial scores, 2 tiles
+constexpr int kOffXOwn = kOffXPeer + 2 * kXBytes;       // own partial scores (fp16), 2 tiles
+constexpr int kOffPMax = kOffXOwn + 2 * kXBytes;        // fp32 [2 pages][2 halves][128] half-row maxima
 constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;      // fp32 [2 items][2 halves][128] half-row sums
 constexpr int kOffBar = kOffLSum + 4 * kRows * 4;
-constexpr int kNumBars = 2 * kStages + 34;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 
-constexpr int kThreads = 448;            // 14 warps: TMA, MMA, 4 exchange, 8 softmax
-constexpr int kXchgWarp0 = 2, kSoftWarp0 = 6;
+constexpr int kThreads = 448;            // 14 warps
+constexpr int kSenderWarp0 = 2, kSoftWarp0 = 6;
 constexpr int kSoftWarps = 8;
 
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemQ = 384, kTmemCols = 512;
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 384, kTmemCols = 512;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 
@@ -90,16 +90,19 @@ struct DecodeParams {
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], s_free[2], p_full[2], p_free[2];
-  uint64_t x_recv[2];    // peer's fp16 partial scores landed in x buffer b (1 arrival + 16 KB tx)
-  uint64_t x_sendok[2];  // peer has consumed its x buffer b, which this CTA may refill (8 remote arrivals)
-  uint64_t o_full, o_free, mma_done, pad;
+  uint64_t s_full;       // QK product of the current page is in S
+  uint64_t s_read;       // the sender has read S (the next QK may overwrite it)
+  uint64_t own_full[2];  // own fp16 partial-score tile b written (4 sender warps)
+  uint64_t own_free[2];  // own tile b consumed by the softmax (8 warps) and read by its bulk copy (1)
+  uint64_t x_recv[2];    // peer's fp16 partial scores landed in tile b (1 arrival + 16 KB tx)
+  uint64_t x_sendok[2];  // peer has consumed its tile b, which this CTA may refill (8 remote arrivals)
+  uint64_t p_full[2];    // P buffer b written (O rescaled if needed), 8 softmax warps
+  uint64_t p_free[2];    // PV product that read P buffer b is complete
+  uint64_t o_full, o_free, qk_done, pad;
   uint64_t pmax[2][4];   // the two softmax warps of row quarter q posted their page-b half-row maxima
   uint64_t lsum[4];      // the two softmax warps of row quarter q posted their half-row sums (per item)
-  uint64_t stg_ok[2];    // send staging tile b may be rewritten (issuer, after the old copy read it)
-  uint64_t stg_full[2];  // send staging tile b written by the 4 sender warps
 };
-static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
+constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 16 + 1024;
 
 __device__ __forceinline__ void report(int32_t* status, int bits) {
   if (status) atomicOr(status, bits);
@@ -108,6 +111,8 @@ __device__ __forceinline__ void report(int32_t* status, int bits) {
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
+// For data a peer CTA wrote with st.async: its complete_tx releases at cluster
+// scope, so the waiter must acquire at cluster scope to see the stores.
 __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
   return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort));
 }
@@ -125,9 +130,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_kv = smem + kOffKV;
   uint8_t* s_qrope = smem + kOffQRope;
-  uint8_t* s_p = smem + kOffP;
-  uint8_t* s_x = smem + kOffX;
-  uint8_t* s_xs = smem + kOffXS;
+  uint8_t* s_xpeer = smem + kOffXPeer;
+  uint8_t* s_xown = smem + kOffXOwn;
   float* s_pmax = reinterpret_cast<float*>(smem + kOffPMax);
   float* s_lsum = reinterpret_cast<float*>(smem + kOffLSum);
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
@@ -154,26 +158,24 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     }
     mbar_init(&bars->q_full, 1 + kSoftWarps);
     mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_read, 4);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 4 + kSoftWarps);
-      mbar_init(&bars->p_full[b], kSoftWarps);
-      mbar_init(&bars->p_free[b], 1);
+      mbar_init(&bars->own_full[b], 4);
+      mbar_init(&bars->own_free[b], kSoftWarps + 1);
       mbar_init(&bars->x_recv[b], 1);
       mbar_init(&bars->x_sendok[b], kSoftWarps);
+      mbar_init(&bars->p_full[b], kSoftWarps);
+      mbar_init(&bars->p_free[b], 1);
     }
     for (int b = 0; b < 2; ++b) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);   // armed for pages 0, 1
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, kSoftWarps);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->qk_done, 1);
     for (int q = 0; q < 4; ++q) {
       mbar_init(&bars->pmax[0][q], 2);
       mbar_init(&bars->pmax[1][q], 2);
       mbar_init(&bars->lsum[q], 2);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->stg_ok[b], 1);
-      mbar_init(&bars->stg_full[b], 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -230,127 +232,144 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // One thread issues both product streams: QK of page qg as soon as its
+    // stage has landed and S has been read out, and PV of page pg (< qg) as
+    // soon as its P is written.  Readiness is polled without blocking, so a
+    // page waiting for its softmax never holds back the next QK.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
       const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
-      const uint32_t kv0 = smem_u32(s_kv), qr0 = smem_u32(s_qrope), p0 = smem_u32(s_p);
-      int g = 0;
-      bool ok = true;
-      auto issue_qk = [&](int gq) -> bool {
-        const int s = gq % kStages, b = gq & 1;
-        if (!mbar_wait(&bars->kv_full[s], (gq / kStages) & 1, abort_flag)) return false;
-        if (gq >= 2 && !mbar_wait(&bars->s_free[b], ((gq >> 1) - 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + kTmemS + 64 * b;
-        const uint32_t st = kv0 + s * kStageBytes;
-#pragma unroll
-        for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16
-          mma_ts(d, tmem + kTmemQ + 8 * t,
-                 sdesc(st + (t >> 2) * kChunkBytes + (t & 3) * 32, 16, 1024, kSwizzle128B), idesc_qk,
-                 t != 0);
-#pragma unroll
-        for (int t = 0; t < 2; ++t)    // RoPE half: K = 32
-          mma_ss(d, sdesc(qr0 + t * 32, 16, 512, kSwizzle64B),
-                 sdesc(st + 4 * kChunkBytes + t * 32, 16, 512, kSwizzle64B), idesc_qk, 1);
-        mma_commit(&bars->s_full[b]);
-        return true;
+      const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
+      const uint64_t kr_desc0 = sdesc(smem_u32(s_kv) + 4 * kChunkBytes, 16, 512, kSwizzle64B);
+      const uint64_t qr_desc = sdesc(smem_u32(s_qrope), 16, 512, kSwizzle64B);
+      const uint64_t v_desc0 = sdesc(smem_u32(s_kv), kChunkBytes, 1024, kSwizzle128B);
+      auto pages_of = [&](int it) {
+        return items[(size_t)it * kItemWords + kItPageEnd] - items[(size_t)it * kItemWords + kItPageBegin];
       };
-      for (int it = it_begin; it < it_end && ok; ++it) {
-        const int32_t* w = items + (size_t)it * kItemWords;
-        const int n = w[kItPageEnd] - w[kItPageBegin];
-        const int ii = it - it_begin;
-        if (!mbar_wait(&bars->q_full, ii & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (!issue_qk(g)) { ok = false; break; }
-        if (n == 1) mma_commit(&bars->q_empty);
-        for (int j = 0; j < n; ++j) {
-          if (j + 1 < n) {
-            if (!issue_qk(g + j + 1)) { ok = false; break; }
-            if (j + 2 == n) mma_commit(&bars->q_empty);
-          }
-          const int gj = g + j, b = gj & 1, s = gj % kStages;
-          if (!mbar_wait(&bars->p_full[b], (gj >> 1) & 1, abort_flag)) { ok = false; break; }
-          if (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t st = kv0 + s * kStageBytes, pb = p0 + b * kPBytes;
+      int q_it = it_begin, q_j = 0, qg = 0, q_n = (it_begin < it_end) ? pages_of(it_begin) : 0;   // QK stream
+      int p_it = it_begin, p_j = 0, pg = 0, p_n = q_n;                                            // PV stream
+      bool ok = true;
+      uint64_t t_last = globaltimer();
+      while (ok && (q_it < it_end || p_it < it_end)) {
+        bool progressed = false;
+        if (q_it < it_end) {
+          const int ii = q_it - it_begin, s = qg % kStages;
+          if ((q_j != 0 || mbar_test(&bars->q_full, ii & 1)) && mbar_test(&bars->kv_full[s], (qg / kStages) & 1) &&
+              (qg == 0 || mbar_test(&bars->s_read, (qg - 1) & 1))) {
+            tc_fence_after();
+            const uint64_t kvd = kv_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+            const uint64_t krd = kr_desc0 + (uint64_t)((s * kStageBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16
-            mma_ss(tmem + kTmemO, sdesc(pb + kk * 32, 16, 1024, kSwizzle128B),
-                   sdesc(st + kk * 2048, kChunkBytes, 1024, kSwizzle128B), idesc_pv, (j | kk) != 0);
-          mma_commit(&bars->p_free[b]);
-          mma_commit(&bars->kv_empty[s]);
-          mma_commit(&bars->o_full);
+            for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16, A = q_lat from TMEM
+              mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * t,
+                     kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)    // RoPE half: K = 32
+              mma_ss(tmem + kTmemS, qr_desc + (uint64_t)(t * 2), krd + (uint64_t)(t * 2), idesc_qk, 1);
+            mma_commit(&bars->s_full);
+            ++qg;
+            if (++q_j == q_n) {
+              mma_commit(&bars->q_empty);
+              q_j = 0;
+              if (++q_it < it_end) q_n = pages_of(q_it);
+            }
+            progressed = true;
+          }
         }
-        g += n;
+        if (p_it < it_end && pg < qg) {
+          const int ii = p_it - it_begin, s = pg % kStages, b = pg & 1;
+          if (mbar_test(&bars->p_full[b], (pg >> 1) & 1) &&
+              (p_j != 0 || ii == 0 || mbar_test(&bars->o_free, (ii - 1) & 1))) {
+            tc_fence_after();
+            const uint64_t vd = v_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16; P (bf16 pairs) from TMEM
+              mma_ts(tmem + kTmemO, tmem + kTmemP + 32 * b + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                     (p_j | kk) != 0);
+            mma_commit(&bars->p_free[b]);
+            mma_commit(&bars->kv_empty[s]);
+            mma_commit(&bars->o_full);
+            ++pg;
+            if (++p_j == p_n) {
+              p_j = 0;
+              if (++p_it < it_end) p_n = pages_of(p_it);
+            }
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          t_last = globaltimer();
+        } else if (*abort_flag || globaltimer() - t_last > kWaitLimitNs) {
+          ok = false;
+        }
       }
       if (!ok) {
         *abort_flag = 1;
         report(p.status, MLA_STATUS_TIMEOUT);
       }
-      mma_commit(&bars->mma_done);
-      mbar_wait(&bars->mma_done, 0, nullptr);   // no MMA may still write TMEM at dealloc
+      mma_commit(&bars->qk_done);
+      mbar_wait(&bars->qk_done, 0, nullptr);   // no MMA may still write TMEM at dealloc
     }
   } else if (warp < kSoftWarp0) {
     // ------------------------------------------------------------ score sender (4 warps)
-    // This CTA's partial scores (its 288 columns), rounded to fp16, go to the
-    // peer's exchange tile b by one bulk copy that completes on the peer's
-    // x_recv[b].  Thread = one row (TMEM lane), 64 keys; the tile is staged
-    // locally with 16-byte chunks XOR-swizzled by (row & 7).
+    // Reads this CTA's partial scores (its 288 columns) as soon as the QK
+    // product lands, frees S, rounds to fp16 into the local own-tile b, and
+    // one thread pushes that tile to the peer's tile b with a bulk copy that
+    // completes on the peer's x_recv[b].  Thread = one row, 64 keys; 16-byte
+    // chunks XOR-swizzled by (row & 7).  (Per-thread st.async stores into
+    // the peer raced with the peer's reads under load; the bulk copy is
+    // deterministic.)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const bool issuer = (warp == 2 && lane == 0);
-    const uint32_t x_peer = mapa(smem_u32(s_x), peer);
+    const uint32_t x_peer = mapa(smem_u32(s_xpeer), peer);
     const uint32_t x_recv_peer = mapa(smem_u32(&bars->x_recv[0]), peer);
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
       const int n = w[kItPageEnd] - w[kItPageBegin];
-      for (int j = 0; j < n; ++j) {
-        const int gj = g + j, b = gj & 1;
+      for (int j = 0; j < n; ++j, ++g) {
+        const int b = g & 1;
         uint32_t v[64];
-        if (!warp_wait(&bars->s_full[b], (gj >> 1) & 1, abort_flag)) goto xchg_fail;
+        if (!warp_wait(&bars->s_full, g & 1, abort_flag)) goto sender_fail;
         tc_fence_after();
-        tmem_ld32(tmem + lane_addr + kTmemS + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(v));
-        tmem_ld32(tmem + lane_addr + kTmemS + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld32(tmem + lane_addr + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tmem + lane_addr + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[b]);
+        if (lane == 0) mbar_arrive(&bars->s_read);
         uint32_t hv[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) hv[k] = pack_f16(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-        // staging tile b is reusable once the copy issued two pages ago has read it
-        if (issuer) {
-          bulk_wait_read<1>();
-          mbar_arrive(&bars->stg_ok[b]);
-        }
-        if (!warp_wait(&bars->stg_ok[b], (gj >> 1) & 1, abort_flag)) goto xchg_fail;
+        if (g >= 2 && !warp_wait(&bars->own_free[b], ((g >> 1) - 1) & 1, abort_flag)) goto sender_fail;
+        if (g >= 2 && !warp_wait(&bars->x_sendok[b], ((g >> 1) - 1) & 1, abort_flag)) goto sender_fail;
         {
-          uint8_t* row = s_xs + b * kXBytes + r * kXRow;
+          uint8_t* own = s_xown + b * kXBytes + r * kXRow;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(row + ((k ^ (r & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(own + ((k ^ (r & 7)) << 4)) =
                 make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
         }
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();   // the bulk copy below reads the tile through the async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->stg_full[b]);
-        if (issuer) {
-          if (!mbar_wait(&bars->stg_full[b], (gj >> 1) & 1, abort_flag)) goto xchg_fail;
-          if (gj >= 2 && !mbar_wait(&bars->x_sendok[b], ((gj >> 1) - 1) & 1, abort_flag)) goto xchg_fail;
-          bulk_copy_to_peer(x_peer + b * kXBytes, smem_u32(s_xs + b * kXBytes), kXBytes, x_recv_peer + 8 * b);
+        if (lane == 0) mbar_arrive(&bars->own_full[b]);
+        if (warp == kSenderWarp0 && lane == 0) {
+          // one bulk copy of the whole tile to the peer, completing on its x_recv[b];
+          // the local tile may be rewritten only after the copy has read it
+          if (!mbar_wait(&bars->own_full[b], (g >> 1) & 1, abort_flag)) goto sender_fail;
+          bulk_copy_to_peer(x_peer + b * kXBytes, smem_u32(s_xown + b * kXBytes), kXBytes, x_recv_peer + 8 * b);
           bulk_commit();
+          bulk_wait_read<0>();
+          mbar_arrive(&bars->own_free[b]);
         }
       }
-      g += n;
     }
-    goto xchg_done;
-  xchg_fail:
+    goto sender_done;
+  sender_fail:
     *abort_flag = 1;
     if (lane == 0) report(p.status, MLA_STATUS_TIMEOUT);
-  xchg_done:
-    if (issuer) bulk_wait_read<0>();   // the staging tiles must outlive their copies
+  sender_done:;
   } else {
     // ------------------------------------------------------------ softmax / epilogue (8 warps)
     // Thread = (row r, key half c): keys [32c, 32c+32) of each page, output
@@ -359,7 +378,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int c = (warp - kSoftWarp0) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    uint8_t* prow0 = s_p + r * 128;
     const float sl2 = p.scale_log2;
     const uint32_t x_sendok_peer = mapa(smem_u32(&bars->x_sendok[0]), peer);
     int g = 0;
@@ -394,41 +412,41 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       for (int j = 0; j < n; ++j) {
         const int gj = g + j, b = gj & 1;
         // full score = fp16(own partial) + fp16(peer partial), identical in both CTAs
-        if (!warp_wait(&bars->x_recv[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
-        if (!warp_wait(&bars->s_full[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
-        tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_addr + kTmemS + 64 * b + 32 * c, v);
-        uint4 pr[4];
+        if (!warp_wait(&bars->own_full[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait_cluster(&bars->x_recv[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
+        uint4 po[4], pr[4];
         {
-          const uint8_t* xrow = s_x + b * kXBytes + r * kXRow;
+          const uint8_t* orow = s_xown + b * kXBytes + r * kXRow;
+          const uint8_t* xrow = s_xpeer + b * kXBytes + r * kXRow;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            pr[k] = *reinterpret_cast<const uint4*>(xrow + (((4 * c + k) ^ (r & 7)) << 4));
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t off = (uint32_t)(((4 * c + k) ^ (r & 7)) << 4);
+            po[k] = *reinterpret_cast<const uint4*>(orow + off);
+            pr[k] = *reinterpret_cast<const uint4*>(xrow + off);
+          }
         }
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free[b]);
+        float sc[32];
         uint32_t used = 0;
         {
+          const uint32_t* ow = reinterpret_cast<const uint32_t*>(po);
           const uint32_t* pw = reinterpret_cast<const uint32_t*>(pr);
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float2 own = round_f16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-            const float2 oth = unpack_f16x2(pw[k]);
-            used |= pw[k];
-            v[2 * k] = __float_as_uint(own.x + oth.x);
-            v[2 * k + 1] = __float_as_uint(own.y + oth.y);
+            const float2 a = unpack_f16x2(ow[k]);
+            const float2 o = unpack_f16x2(pw[k]);
+            used |= pw[k] ^ ow[k];
+            sc[2 * k] = a.x + o.x;
+            sc[2 * k + 1] = a.y + o.y;
           }
         }
-        // exchange tile b is consumed: re-arm it for page gj + 2, then let the peer refill it
+        // both tiles b are consumed: re-arm x_recv[b] for page gj + 2, then release the tiles
         {
           uint32_t ok_addr = x_sendok_peer + 8 * b;
-          asm volatile("" : "+r"(ok_addr) : "r"(used));   // issue only after the tile was read
+          asm volatile("" : "+r"(ok_addr) : "r"(used));   // issue only after the tiles were read
           __syncwarp();
           if (lane == 0) {
             if (warp == kSoftWarp0) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);
+            mbar_arrive(&bars->own_free[b]);
             mbar_arrive_relaxed_cluster(ok_addr);
           }
         }
@@ -436,11 +454,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (tok0 + 32 > kv_len) {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
-            if (tok0 + k >= kv_len) v[k] = __float_as_uint(-CUDART_INF_F);
+            if (tok0 + k >= kv_len) sc[k] = -CUDART_INF_F;
         }
-        float mloc = __uint_as_float(v[0]);
+        float mloc;
+        {
+          float t[16];
 #pragma unroll
-        for (int k = 1; k < 32; ++k) mloc = fmaxf(mloc, __uint_as_float(v[k]));
+          for (int k = 0; k < 16; ++k) t[k] = fmaxf(sc[k], sc[k + 16]);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) t[k] = fmaxf(t[k], t[k + 8]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) t[k] = fmaxf(t[k], t[k + 4]);
+          mloc = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
+        }
         s_pmax[(b * 2 + c) * kRows + r] = mloc;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->pmax[b][quarter]);
@@ -458,16 +484,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         }
         const float nb = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
         uint32_t pk[16];
-        float ps = 0.f;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float e0 = ex2(fmaf(__uint_as_float(v[2 * k]), sl2, nb));
-          const float e1 = ex2(fmaf(__uint_as_float(v[2 * k + 1]), sl2, nb));
+          const float e0 = ex2(fmaf(sc[2 * k], sl2, nb));
+          const float e1 = ex2(fmaf(sc[2 * k + 1], sl2, nb));
           pk[k] = pack_bf16(e0, e1);
-          ps += e0 + e1;
+          ps[k & 3] += e0 + e1;
         }
-        l_run = l_run * alpha + ps;
+        l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
+        // P buffer b is free once the PV product two pages back has completed
         if (gj >= 2 && !warp_wait(&bars->p_free[b], ((gj >> 1) - 1) & 1, abort_flag)) goto softmax_fail;
         if (__any_sync(0xffffffffu, move && j > 0)) {
           if (!warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
@@ -484,14 +511,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           }
           tmem_st_wait();
         }
-        {
-          uint8_t* prow = prow0 + b * kPBytes;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(prow + (((4 * c + k) ^ (r & 7)) << 4)) =
-                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
-        }
-        fence_proxy_async_smem();
+        tmem_st16(tmem + lane_addr + kTmemP + 32 * b + 16 * c, pk);   // keys [32c, 32c+32) as bf16 pairs
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->p_full[b]);
