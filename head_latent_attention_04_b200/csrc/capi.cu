@@ -195,6 +195,29 @@ mla_status_t mla_combine(const mla_dims_t* dims, const void* plan_dev, const flo
                         lse_part, o_lat, lse_out, stream);
 }
 
+mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                                              const void* kv_pool, const int32_t* block_table,
+                                              const int32_t* seq_lens, const void* plan_host,
+                                              size_t plan_bytes, int32_t num_clusters, void* o_lat,
+                                              float* lse_out, int32_t* status, void* stream) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  MLA_TRY(check_ptr(q_rope, "q_rope"));
+  MLA_TRY(check_ptr(kv_pool, "kv_pool"));
+  MLA_TRY(check_ptr(block_table, "block_table"));
+  MLA_TRY(check_ptr(seq_lens, "seq_lens"));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  if (!plan_host || (reinterpret_cast<uintptr_t>(plan_host) & 3u))
+    return set_error(MLA_ERR_INVALID_ARG, "plan_host is NULL or not 4-byte aligned");
+  if (num_clusters < 1 || num_clusters > 4096)
+    return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
+  return decode_attn_combine_noalloc(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_host,
+                                     plan_bytes, num_clusters, o_lat, lse_out, status, stream);
+}
+
+size_t mla_noalloc_scratch_bytes(void) { return noalloc_scratch_bytes(); }
+
 mla_status_t mla_debug_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
                                     int32_t n_pages, int32_t max_blocks_per_seq, int32_t num_blocks,
                                     void* out, int32_t* status, void* stream) {

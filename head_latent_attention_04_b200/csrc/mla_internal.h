@@ -2,6 +2,7 @@
 #pragma once
 #include "../../include/mla.h"
 
+#include <stddef.h>
 #include <stdint.h>
 
 namespace mla {
@@ -30,5 +31,11 @@ mla_status_t launch_gather_pages(const void* kv_pool, const int32_t* block_table
                                  int32_t n_pages, int32_t max_blocks, int32_t num_blocks, void* out,
                                  int32_t* status, void* stream);
 mla_status_t decode_max_clusters(int32_t* n);
+mla_status_t decode_attn_combine_noalloc(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+                                         const void* kv_pool, const int32_t* block_table,
+                                         const int32_t* seq_lens, const void* plan_host,
+                                         size_t plan_bytes, int32_t num_clusters, void* o_lat,
+                                         float* lse_out, int32_t* status, void* stream);
+size_t noalloc_scratch_bytes();
 
 }  // namespace mla

@@ -26,7 +26,7 @@ MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_TIMEOUT = 3, 4, 5
 STATUS_BAD_BLOCK, STATUS_TIMEOUT, STATUS_BAD_SEQLEN = 0x1, 0x2, 0x4
 EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
-           "mla_debug_gather_pages")
+           "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes")
 
 
 class MlaDims(ctypes.Structure):
@@ -50,9 +50,14 @@ for _name, _args in {
     "mla_decode_attn": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_combine": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_debug_gather_pages": [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
+    "mla_decode_attn_combine_noalloc": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _vp, _vp, _vp, _vp],
 }.items():
     getattr(_lib, _name).argtypes = _args
     getattr(_lib, _name).restype = _i32
+
+
+_lib.mla_noalloc_scratch_bytes.argtypes = []
+_lib.mla_noalloc_scratch_bytes.restype = _sz
 
 
 class MlaError(RuntimeError):
@@ -143,6 +148,27 @@ def decode_attn(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_dev, n
 def combine(dims, plan_dev, o_part, lse_part, o_lat, lse_out=None, stream=None):
     _check(_lib.mla_combine(ctypes.byref(dims), _ptr(plan_dev), _ptr(o_part), _ptr(lse_part),
                             _ptr(o_lat), _ptr(lse_out), _stream(stream)), "mla_combine")
+
+
+def noalloc_scratch_bytes() -> int:
+    """Size of the library-owned device array used by ``decode_attn_combine_noalloc``."""
+    return _lib.mla_noalloc_scratch_bytes()
+
+
+def decode_attn_combine_noalloc(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_host: np.ndarray,
+                                num_clusters, o_lat, lse_out=None, status=None, stream=None):
+    """Attention + split merge with no caller workspace and no device allocation.
+
+    For callers that may not allocate device memory (e.g. a runtime that has
+    pre-reserved HBM for its KV cache): ``plan_host`` is the host plan from
+    :func:`plan`; the plan copy and the partial outputs live in a fixed array
+    inside the library (see :func:`noalloc_scratch_bytes`).
+    """
+    pl = np.ascontiguousarray(plan_host, dtype=np.int32)
+    _check(_lib.mla_decode_attn_combine_noalloc(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(kv_pool),
+                                                _ptr(block_table), _ptr(seq_lens), pl.ctypes.data, pl.nbytes,
+                                                num_clusters, _ptr(o_lat), _ptr(lse_out), _ptr(status),
+                                                _stream(stream)), "mla_decode_attn_combine_noalloc")
 
 
 def debug_gather_pages(kv_pool, block_table, b, n_pages, max_blocks, num_blocks, out, status=None,

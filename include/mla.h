@@ -161,6 +161,41 @@ mla_status_t mla_combine(const mla_dims_t* dims, const void* plan_dev, const flo
                          float* lse_out, void* stream);
 
 /*
+ * mla_decode_attn_combine_noalloc -- mla_decode_attn followed by mla_combine,
+ * for callers that cannot allocate device memory.  There is no counterpart in
+ * the paper; it exists for deployment.
+ *
+ * Some callers may not call cudaMalloc while they run: a serving runtime that
+ * reserves nearly all HBM for its paged KV-cache pool at start-up and only
+ * hands kernels buffers it planned for, or a plugin invoked where allocation
+ * is forbidden.  Such a caller cannot supply the o_part / lse_part workspace
+ * or a device copy of the plan that the two calls above take.  This entry
+ * point takes the HOST plan (from mla_plan) and keeps the plan copy and the
+ * split-KV partial outputs in a fixed device array owned by the library:
+ *   - its size is mla_noalloc_scratch_bytes() (32 MiB); a batch whose plan
+ *     needs more returns MLA_ERR_WORKSPACE_TOO_SMALL and launches nothing;
+ *   - every GPU that loads the library holds that array until the process
+ *     exits;
+ *   - the first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture;
+ *   - it allocates nothing and frees nothing;
+ *   - all calls share the array, and it keeps the last call's contents
+ *     (nothing in it needs to start at zero); calls that overlap on the GPU
+ *     race on it, so serialise them.
+ * The other arguments mean what they mean for mla_decode_attn / mla_combine;
+ * o_lat (and lse_out if non-NULL) receive the finished rows.
+ */
+mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void* q_lat,
+                                             const void* q_rope, const void* kv_pool,
+                                             const int32_t* block_table, const int32_t* seq_lens,
+                                             const void* plan_host, size_t plan_bytes,
+                                             int32_t num_clusters, void* o_lat, float* lse_out,
+                                             int32_t* status, void* stream);
+
+/* Size in bytes of the device array mla_decode_attn_combine_noalloc works in. */
+size_t mla_noalloc_scratch_bytes(void);
+
+/*
  * mla_debug_gather_pages -- copies the cache rows of sequence b, in token
  * order, through block_table into out bf16 [n_pages*64][576] (bit-exact page
  * indexing check; not on the decode path).  Out-of-range block ids set

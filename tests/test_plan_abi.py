@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_library_exports_every_declared_symbol():
     header = open(os.path.join(ROOT, "include", "mla.h")).read()
-    declared = set(re.findall(r"^\s*(?:mla_status_t|int32_t|const char\*)\s+(mla_\w+)\s*\(", header, re.M))
+    declared = set(re.findall(r"^\s*(?:mla_status_t|int32_t|size_t|const char\*)\s+(mla_\w+)\s*\(", header, re.M))
     assert declared == set(mla.EXPORTS)
     lib = ctypes.CDLL(mla._LIB_PATH)
     for name in declared:
