@@ -253,13 +253,13 @@ def workload_config(name, w):
 
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
-    from head_latent_attention_04_b200 import mla
+    from head_latent_attention_04_b200 import dp, mla
     from head_latent_attention_04_b200 import workloads as W
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     preset = W.PRESETS[args.config]
-    w = W.preset_workload(args.config, device=dev, seed=preset.seed + 1000 * rank)
+    w = W.preset_workload(args.config, device=dev, seed=dp.replica_seed(preset.seed, rank))
     acc = algorithmic(w.seq_lens, w.s_q, w.n_heads)
     bt = torch.as_tensor(w.block_table, device=dev)
     dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev)
@@ -346,15 +346,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e2e_local = statistics.fmean(a.elapsed_time(b) for a, b in ee)
     status = int(dec.status.item())
 
-    if world > 1:
-        t = torch.tensor([ms_local, attn_local, e2e_local], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, attn, e2e = t.tolist()
-        st = torch.tensor([status], dtype=torch.int32, device=dev)
-        torch.distributed.all_reduce(st, op=torch.distributed.ReduceOp.MAX)
-        status = int(st.item())
-    else:
-        ms, attn, e2e = ms_local, attn_local, e2e_local
+    # bookkeeping collectives only (identity at one rank): max over ranks, status OR
+    ms, attn, e2e = dp.reduce_max([ms_local, attn_local, e2e_local], device=dev)
+    status = dp.reduce_status(status, device=dev)
     used_graph = graph is not None
     del graph
     if rank != 0:
