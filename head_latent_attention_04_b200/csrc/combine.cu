@@ -4,10 +4,18 @@
 // outputs O_i and natural-log LSEs lse_i.  Softmax over the union of the
 // pieces' keys is
 //   L = log sum_i exp(lse_i),   o = sum_i exp(lse_i - L) O_i,
-// the identity the oracle's split-merge pin checks.  HBM-bound: one warp per
-// (row, head) reads m x 512 fp32 with 16-byte loads and writes 512 bf16.
+// the identity the oracle's split-merge pin checks.
+//
+// The pieces live in the column-group-major workspace the attention kernel
+// writes: element (slot, h, col) of O_i sits at
+//   ((slot * 128 + col / 4) * n_heads + h) * 4 + col % 4,
+// so that 32 consecutive heads of one 4-column group are 512 contiguous bytes.
+// HBM-bound: a block takes one row and 32 columns; thread (h, half) reads 4
+// column groups of every piece (consecutive h -> coalesced 16-byte loads) and
+// writes 16 bf16 of its head (one full 32-byte sector).
 #include "mla_internal.h"
 #include "plan_format.h"
+#include "ptx.cuh"
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
@@ -15,52 +23,51 @@
 namespace mla {
 namespace {
 
+constexpr int kCombineThreads = 256;   // 128 heads x 2 column halves
+constexpr int kCombineCols = 32;       // columns per block
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kCombineThreads)
 mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o_part,
                    const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o_lat,
                    float* __restrict__ lse_out, int n_heads) {
   const int n = blockIdx.x;
-  const int h = blockIdx.y * 4 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
+  const int h = threadIdx.x & 127;
+  const int half = threadIdx.x >> 7;
   if (h >= n_heads) return;
   const int32_t* rs = plan + plan[kHdrOffRows];
   const int s0 = rs[n], s1 = rs[n + 1];
   if (s1 <= s0) return;   // row written whole by the attention kernel
 
   float lmax = -CUDART_INF_F;
-  for (int s = s0; s < s1; ++s) lmax = fmaxf(lmax, lse_part[(size_t)s * n_heads + h]);
+  for (int s = s0; s < s1; ++s) lmax = fmaxf(lmax, __ldg(lse_part + (size_t)s * n_heads + h));
   float z = 0.f;
   for (int s = s0; s < s1; ++s) {
-    const float l = lse_part[(size_t)s * n_heads + h];
+    const float l = __ldg(lse_part + (size_t)s * n_heads + h);
     z += (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax);
   }
   const float inv_z = z > 0.f ? 1.f / z : 0.f;
 
+  const int g0 = blockIdx.y * (kCombineCols / 4) + half * 4;   // first of this thread's 4 column groups
   float4 acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s = s0; s < s1; ++s) {
-    const float l = lse_part[(size_t)s * n_heads + h];
+    const float l = __ldg(lse_part + (size_t)s * n_heads + h);
     const float wgt = (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax) * inv_z;
-    const float4* src = reinterpret_cast<const float4*>(o_part + ((size_t)s * n_heads + h) * 512);
+    const float4* src = reinterpret_cast<const float4*>(o_part) + ((size_t)s * 128 + g0) * n_heads + h;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const float4 v = __ldg(src + k * 32 + lane);
+      const float4 v = __ldg(src + (size_t)k * n_heads);
       acc[k].x += wgt * v.x; acc[k].y += wgt * v.y; acc[k].z += wgt * v.z; acc[k].w += wgt * v.w;
     }
   }
-  __nv_bfloat16* dst = o_lat + ((size_t)n * n_heads + h) * 512;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    __nv_bfloat162 a = __floats2bfloat162_rn(acc[k].x, acc[k].y);
-    __nv_bfloat162 b = __floats2bfloat162_rn(acc[k].z, acc[k].w);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t*>(&a);
-    u.y = *reinterpret_cast<uint32_t*>(&b);
-    *reinterpret_cast<uint2*>(dst + (k * 32 + lane) * 4) = u;
-  }
-  if (lse_out && lane == 0) lse_out[(size_t)n * n_heads + h] = z > 0.f ? lmax + __logf(z) : -CUDART_INF_F;
+  uint4* dst = reinterpret_cast<uint4*>(o_lat + ((size_t)n * n_heads + h) * 512 + 4 * g0);
+  dst[0] = make_uint4(ptx::pack_bf16(acc[0].x, acc[0].y), ptx::pack_bf16(acc[0].z, acc[0].w),
+                      ptx::pack_bf16(acc[1].x, acc[1].y), ptx::pack_bf16(acc[1].z, acc[1].w));
+  dst[1] = make_uint4(ptx::pack_bf16(acc[2].x, acc[2].y), ptx::pack_bf16(acc[2].z, acc[2].w),
+                      ptx::pack_bf16(acc[3].x, acc[3].y), ptx::pack_bf16(acc[3].z, acc[3].w));
+  if (lse_out && blockIdx.y == 0 && half == 0)
+    lse_out[(size_t)n * n_heads + h] = z > 0.f ? lmax + __logf(z) : -CUDART_INF_F;
 }
 
 __global__ void mla_gather_pages_kernel(const uint4* __restrict__ pool, const int32_t* __restrict__ bt,
@@ -81,8 +88,8 @@ __global__ void mla_gather_pages_kernel(const uint4* __restrict__ pool, const in
 mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,
                             const float* o_part, const float* lse_part, void* o_lat,
                             float* lse_out, void* stream) {
-  dim3 grid(n_rows, (d.n_heads + 3) / 4);
-  mla_combine_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+  dim3 grid(n_rows, 512 / kCombineCols);
+  mla_combine_kernel<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse_out, d.n_heads);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));

@@ -26,11 +26,12 @@
 // the sender has read it), P [320,384) as two bf16 buffers (A operand of the
 // PV product), q_lat half [384,512) as bf16 pairs (A operand of QK).
 //
-// Warp roles (448 threads): warp 0 TMA producer; warp 1 MMA issuer and TMEM
-// owner (one thread, polling the QK and PV streams so neither blocks the
-// other); warps 2-5 score sender (one thread per row, 64 keys); warps 6-13
-// softmax / correction / epilogue (two warps per TMEM lane quarter, one per
-// 32-key half).  The grid
+// Warp roles (480 threads): warp 0 TMA producer; warp 1 QK issuer and TMEM
+// owner; warp 2 PV issuer (two issuing threads, so a page waiting for its
+// softmax never holds back the next QK, and the tensor pipe takes work from
+// both); warps 3-6 score sender and q_lat loader (one thread per row);
+// warps 7-14 softmax / correction / epilogue (two warps per TMEM lane
+// quarter, one per 32-key half).  The grid
 // is persistent: one cluster per SM pair, each walking the (row, page range)
 // items the host plan gives it.  Every wait is bounded (ptx::kWaitLimitNs);
 // on expiry the CTA sets MLA_STATUS_TIMEOUT and unwinds without trapping.
@@ -65,8 +66,8 @@ constexpr int kOffPMax = kOffXOwn + 2 * kXBytes;        // fp32 [2 pages][2 halv
 constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;      // fp32 [2 items][2 halves][128] half-row sums
 constexpr int kOffBar = kOffLSum + 4 * kRows * 4;
 
-constexpr int kThreads = 448;            // 14 warps
-constexpr int kSenderWarp0 = 2, kSoftWarp0 = 6;
+constexpr int kThreads = 480;            // 15 warps
+constexpr int kSenderWarp0 = 3, kSoftWarp0 = 7;
 constexpr int kSoftWarps = 8;
 
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 384, kTmemCols = 512;
@@ -98,7 +99,7 @@ struct Bars {
   uint64_t x_sendok[2];  // peer has consumed its tile b, which this CTA may refill (8 remote arrivals)
   uint64_t p_full[2];    // P buffer b written (O rescaled if needed), 8 softmax warps
   uint64_t p_free[2];    // PV product that read P buffer b is complete
-  uint64_t o_full, o_free, qk_done, pad;
+  uint64_t o_full, o_free, qk_done, pv_done;
   uint64_t pmax[2][4];   // the two softmax warps of row quarter q posted their page-b half-row maxima
   uint64_t lsum[4];      // the two softmax warps of row quarter q posted their half-row sums (per item)
 };
@@ -156,7 +157,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->q_full, 1 + kSoftWarps);
+    mbar_init(&bars->q_full, 1 + 4);   // q_rope TMA + the 4 q_lat loader warps
     mbar_init(&bars->q_empty, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_read, 4);
@@ -172,6 +173,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_free, kSoftWarps);
     mbar_init(&bars->qk_done, 1);
+    mbar_init(&bars->pv_done, 1);
     for (int q = 0; q < 4; ++q) {
       mbar_init(&bars->pmax[0][q], 2);
       mbar_init(&bars->pmax[1][q], 2);
@@ -204,6 +206,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (ii > 0 && !mbar_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto producer_fail;
         mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
         tma_load_3d(s_qrope, &tm_qrope, &bars->q_full, 32 * rank, 0, row);
+        if (it + 1 < it_end)   // the next item's q_lat rows, so that its loader reads them from L2
+          bulk_prefetch_l2(p.q_lat + (size_t)items[(size_t)(it + 1) * kItemWords + kItRow] * p.n_heads * 512,
+                           (uint32_t)p.n_heads * 1024u);
         for (int pg = w[kItPageBegin]; pg < w[kItPageEnd]; ++pg, ++g) {
           const int s = g % kStages;
           if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, abort_flag))
@@ -231,77 +236,42 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         mbar_wait(&bars->kv_full[k % kStages], (k / kStages) & 1, nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // One thread issues both product streams: QK of page qg as soon as its
-    // stage has landed and S has been read out, and PV of page pg (< qg) as
-    // soon as its P is written.  Readiness is polled without blocking, so a
-    // page waiting for its softmax never holds back the next QK.
+    // ------------------------------------------------------------ QK issuer
+    // S = [q_lat | q_rope] . [c_KV | k_rope]^T over this CTA's 288 columns:
+    // M = 128 rows, N = 64 keys, 16 MMAs with A = q_lat from TMEM and 2 with
+    // A = q_rope from shared memory.  S is single-buffered; the sender frees
+    // it (s_read) as soon as it has copied the product out.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
       const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
       const uint64_t kr_desc0 = sdesc(smem_u32(s_kv) + 4 * kChunkBytes, 16, 512, kSwizzle64B);
       const uint64_t qr_desc = sdesc(smem_u32(s_qrope), 16, 512, kSwizzle64B);
-      const uint64_t v_desc0 = sdesc(smem_u32(s_kv), kChunkBytes, 1024, kSwizzle128B);
-      auto pages_of = [&](int it) {
-        return items[(size_t)it * kItemWords + kItPageEnd] - items[(size_t)it * kItemWords + kItPageBegin];
-      };
-      int q_it = it_begin, q_j = 0, qg = 0, q_n = (it_begin < it_end) ? pages_of(it_begin) : 0;   // QK stream
-      int p_it = it_begin, p_j = 0, pg = 0, p_n = q_n;                                            // PV stream
       bool ok = true;
-      uint64_t t_last = globaltimer();
-      while (ok && (q_it < it_end || p_it < it_end)) {
-        bool progressed = false;
-        if (q_it < it_end) {
-          const int ii = q_it - it_begin, s = qg % kStages;
-          if ((q_j != 0 || mbar_test(&bars->q_full, ii & 1)) && mbar_test(&bars->kv_full[s], (qg / kStages) & 1) &&
-              (qg == 0 || mbar_test(&bars->s_read, (qg - 1) & 1))) {
-            tc_fence_after();
-            const uint64_t kvd = kv_desc0 + (uint64_t)((s * kStageBytes) >> 4);
-            const uint64_t krd = kr_desc0 + (uint64_t)((s * kStageBytes) >> 4);
-#pragma unroll
-            for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16, A = q_lat from TMEM
-              mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * t,
-                     kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
-#pragma unroll
-            for (int t = 0; t < 2; ++t)    // RoPE half: K = 32
-              mma_ss(tmem + kTmemS, qr_desc + (uint64_t)(t * 2), krd + (uint64_t)(t * 2), idesc_qk, 1);
-            mma_commit(&bars->s_full);
-            ++qg;
-            if (++q_j == q_n) {
-              mma_commit(&bars->q_empty);
-              q_j = 0;
-              if (++q_it < it_end) q_n = pages_of(q_it);
-            }
-            progressed = true;
+      int g = 0;
+      for (int it = it_begin; ok && it < it_end; ++it) {
+        const int32_t* w = items + (size_t)it * kItemWords;
+        const int n = w[kItPageEnd] - w[kItPageBegin];
+        if (!mbar_wait(&bars->q_full, (it - it_begin) & 1, abort_flag)) { ok = false; break; }
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = g % kStages;
+          if (!mbar_wait(&bars->kv_full[s], (g / kStages) & 1, abort_flag) ||
+              (g > 0 && !mbar_wait(&bars->s_read, (g - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
           }
-        }
-        if (p_it < it_end && pg < qg) {
-          const int ii = p_it - it_begin, s = pg % kStages, b = pg & 1;
-          if (mbar_test(&bars->p_full[b], (pg >> 1) & 1) &&
-              (p_j != 0 || ii == 0 || mbar_test(&bars->o_free, (ii - 1) & 1))) {
-            tc_fence_after();
-            const uint64_t vd = v_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+          tc_fence_after();
+          const uint64_t kvd = kv_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+          const uint64_t krd = kr_desc0 + (uint64_t)((s * kStageBytes) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16; P (bf16 pairs) from TMEM
-              mma_ts(tmem + kTmemO, tmem + kTmemP + 32 * b + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
-                     (p_j | kk) != 0);
-            mma_commit(&bars->p_free[b]);
-            mma_commit(&bars->kv_empty[s]);
-            mma_commit(&bars->o_full);
-            ++pg;
-            if (++p_j == p_n) {
-              p_j = 0;
-              if (++p_it < it_end) p_n = pages_of(p_it);
-            }
-            progressed = true;
-          }
+          for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16, A = q_lat from TMEM
+            mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * t,
+                   kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
+#pragma unroll
+          for (int t = 0; t < 2; ++t)    // RoPE half: K = 32
+            mma_ss(tmem + kTmemS, qr_desc + (uint64_t)(t * 2), krd + (uint64_t)(t * 2), idesc_qk, 1);
+          mma_commit(&bars->s_full);
         }
-        if (progressed) {
-          t_last = globaltimer();
-        } else if (*abort_flag || globaltimer() - t_last > kWaitLimitNs) {
-          ok = false;
-        }
+        if (ok) mma_commit(&bars->q_empty);   // q_lat (TMEM) and q_rope (smem) may be replaced
       }
       if (!ok) {
         *abort_flag = 1;
@@ -310,8 +280,49 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mma_commit(&bars->qk_done);
       mbar_wait(&bars->qk_done, 0, nullptr);   // no MMA may still write TMEM at dealloc
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer
+    // O += P . c_KV: M = 128 rows, N = 256 latent columns, K = 64 keys in 4
+    // MMAs, A = P (bf16 pairs) from TMEM, B = the stage's c_KV half (MN-major).
+    if (lane == 0) {
+      const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+      const uint64_t v_desc0 = sdesc(smem_u32(s_kv), kChunkBytes, 1024, kSwizzle128B);
+      bool ok = true;
+      int g = 0;
+      for (int it = it_begin; ok && it < it_end; ++it) {
+        const int32_t* w = items + (size_t)it * kItemWords;
+        const int n = w[kItPageEnd] - w[kItPageBegin];
+        const int ii = it - it_begin;
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = g % kStages, b = g & 1;
+          if (!mbar_wait(&bars->p_full[b], (g >> 1) & 1, abort_flag) ||
+              (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t vd = v_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16; P (bf16 pairs) from TMEM
+            mma_ts(tmem + kTmemO, tmem + kTmemP + 32 * b + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                   (j | kk) != 0);
+          mma_commit(&bars->p_free[b]);
+          mma_commit(&bars->kv_empty[s]);
+          mma_commit(&bars->o_full);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report(p.status, MLA_STATUS_TIMEOUT);
+      }
+      mma_commit(&bars->pv_done);
+      mbar_wait(&bars->pv_done, 0, nullptr);
+    }
   } else if (warp < kSoftWarp0) {
-    // ------------------------------------------------------------ score sender (4 warps)
+    // ------------------------------------------------------------ q_lat loader and score sender (4 warps)
+    // At each item start the thread of row r copies its 256 q_lat columns
+    // into TMEM (A operand of the QK product) once the previous item's last
+    // QK has completed; the producer has prefetched those rows into L2.
     // Reads this CTA's partial scores (its 288 columns) as soon as the QK
     // product lands, frees S, rounds to fp16 into the local own-tile b, and
     // one thread pushes that tile to the peer's tile b with a bulk copy that
@@ -328,6 +339,27 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
       const int n = w[kItPageEnd] - w[kItPageBegin];
+      const int ii = it - it_begin;
+      if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto sender_fail;
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)w[kItRow] * p.n_heads + r) * 512 +
+                                                          256 * rank);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t v[64];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint4 q = r < p.n_heads ? __ldg(src + 16 * hh + k) : make_uint4(0, 0, 0, 0);
+            v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
+          }
+          tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_full);
+      }
       for (int j = 0; j < n; ++j, ++g) {
         const int b = g & 1;
         uint32_t v[64];
@@ -386,27 +418,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       const int row = w[kItRow], pb = w[kItPageBegin], n = w[kItPageEnd] - pb, slot = w[kItSlot];
       const int kv_len = w[kItKvLen];
       const int ii = it - it_begin;
-
-      // this thread's 128 q_lat columns -> TMEM (bf16 pairs, A operand of the QK product)
-      if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto softmax_fail;
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)row * p.n_heads + r) * 512 +
-                                                          256 * rank + 128 * c);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t v[32];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint4 q = r < p.n_heads ? __ldg(src + h * 8 + k) : make_uint4(0, 0, 0, 0);
-            v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
-          }
-          tmem_st32(tmem + lane_addr + kTmemQ + 64 * c + 32 * h, v);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->q_full);
-      }
 
       float m_ref = -CUDART_INF_F, l_run = 0.f;
       for (int j = 0; j < n; ++j) {
@@ -547,10 +558,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
                                   pack_bf16(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
                                   pack_bf16(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
           } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_part + ((size_t)slot * p.n_heads + r) * 512 + col);
+            // column-group-major partials: a warp's 32 rows of one 4-column group are contiguous
+            float4* dst = reinterpret_cast<float4*>(p.o_part) + ((size_t)slot * 128 + col / 4) * p.n_heads + r;
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-              dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+              dst[(size_t)k * p.n_heads] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
                                    __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
           }
         }

@@ -203,6 +203,14 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
       "r"(src_smem), "r"(bytes), "r"(bar_cluster)
       : "memory");
 }
+// Hint: bring [gptr, gptr + bytes) into L2 (16-byte aligned, multiple of 16 bytes), in 16 KB pieces.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* gptr, uint32_t bytes) {
+  const char* c = static_cast<const char*>(gptr);
+  for (uint32_t off = 0; off < bytes; off += 16384u) {
+    const uint32_t n = bytes - off < 16384u ? bytes - off : 16384u;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c + off), "r"(n) : "memory");
+  }
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed bulk-copy groups still have to read their source.
 template <int N>
@@ -349,8 +357,9 @@ __device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
 __device__ __forceinline__ float2 round_f16x2(float lo, float hi) { return unpack_f16x2(pack_f16(lo, hi)); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
-  return *reinterpret_cast<uint32_t*>(&v);
+  uint32_t r;   // low 16 bits = lo, high 16 bits = hi, each rounded to nearest even
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 }  // namespace ptx

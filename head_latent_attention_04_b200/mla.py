@@ -207,7 +207,7 @@ class Decoder:
         self.plan_dev = torch.from_numpy(self.plan_host).to(dev)
         self.seq_lens_dev = torch.from_numpy(self.seq_lens_host).to(dev)
         slots = max(self.num_slots, 1)
-        self.o_part = torch.empty((slots, n_heads, 512), dtype=torch.float32, device=dev)
+        self.o_part = torch.empty(slots * n_heads * 512, dtype=torch.float32, device=dev)   # internal layout
         self.lse_part = torch.empty((slots, n_heads), dtype=torch.float32, device=dev)
         self.q_lat = torch.empty((self.N, n_heads, 512), dtype=torch.bfloat16, device=dev)
         self.o_lat = torch.empty((self.N, n_heads, 512), dtype=torch.bfloat16, device=dev)

@@ -111,7 +111,7 @@ mla_status_t mla_out_uv(const void* o_lat, const void* w_uv, void* out,
  * ones.  Pieces of a split row are merged by mla_combine.
  *
  * mla_plan_size: upper bounds for the plan (int32 words, in bytes) and for
- *   the two workspace arrays, o_part fp32 [slots][n_heads][512] and
+ *   the two workspace arrays, o_part (slots x n_heads x 512 fp32) and
  *   lse_part fp32 [slots][n_heads], for `num_clusters` clusters.
  * mla_plan: writes the plan into caller memory `plan_host` (plan_bytes from
  *   mla_plan_size); the caller copies it to the device unchanged.  Fails with
@@ -138,7 +138,9 @@ mla_status_t mla_plan(const mla_dims_t* dims, const int32_t* seq_lens_host, int3
  *   seq_lens     int32 [B]  T_b, counting the s_q new tokens (checked against the plan)
  *   plan_dev     the plan from mla_plan, copied to the device
  *   num_clusters the num_clusters the plan was built for (grid = 2 * num_clusters CTAs)
- *   o_part       fp32 [slots][n_heads][512]   workspace (split rows)
+ *   o_part       fp32, slots x n_heads x 512  workspace (split rows); element
+ *                (slot, h, col) at ((slot*128 + col/4)*n_heads + h)*4 + col%4,
+ *                so that the stores of 32 rows are contiguous
  *   lse_part     fp32 [slots][n_heads]        workspace
  *   o_lat        bf16 [N][n_heads][512]       rows not split are written here
  *   lse_out      fp32 [N][n_heads] or NULL    natural-log LSE of the scaled logits
