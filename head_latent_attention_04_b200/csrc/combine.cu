@@ -10,9 +10,10 @@
 // writes: element (slot, h, col) of O_i sits at
 //   ((slot * 128 + col / 4) * n_heads + h) * 4 + col % 4,
 // so that 32 consecutive heads of one 4-column group are 512 contiguous bytes.
-// HBM-bound: a block takes one row and 32 columns; thread (h, half) reads 4
-// column groups of every piece (consecutive h -> coalesced 16-byte loads) and
-// writes 16 bf16 of its head (one full 32-byte sector).
+// HBM-bound: a block takes one row and 16 columns; thread (h, group) reads one
+// 4-column group of every piece (consecutive h -> coalesced 16-byte loads) and
+// writes 4 bf16 of its head.  Small grids (few rows cut into many pieces) still
+// get N x 32 blocks, and each thread's loads over the pieces are independent.
 #include "mla_internal.h"
 #include "plan_format.h"
 #include "ptx.cuh"
@@ -23,8 +24,8 @@
 namespace mla {
 namespace {
 
-constexpr int kCombineThreads = 256;   // 128 heads x 2 column halves
-constexpr int kCombineCols = 32;       // columns per block
+constexpr int kCombineThreads = 512;   // 128 heads x 4 column groups
+constexpr int kCombineCols = 16;       // columns per block
 
 __global__ void __launch_bounds__(kCombineThreads)
 mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o_part,
@@ -32,7 +33,7 @@ mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o
                    float* __restrict__ lse_out, int n_heads) {
   const int n = blockIdx.x;
   const int h = threadIdx.x & 127;
-  const int half = threadIdx.x >> 7;
+  const int grp = threadIdx.x >> 7;
   if (h >= n_heads) return;
   const int32_t* rs = plan + plan[kHdrOffRows];
   const int s0 = rs[n], s1 = rs[n + 1];
@@ -47,26 +48,18 @@ mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o
   }
   const float inv_z = z > 0.f ? 1.f / z : 0.f;
 
-  const int g0 = blockIdx.y * (kCombineCols / 4) + half * 4;   // first of this thread's 4 column groups
-  float4 acc[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int g = blockIdx.y * (kCombineCols / 4) + grp;   // this thread's 4-column group
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
   for (int s = s0; s < s1; ++s) {
     const float l = __ldg(lse_part + (size_t)s * n_heads + h);
     const float wgt = (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax) * inv_z;
-    const float4* src = reinterpret_cast<const float4*>(o_part) + ((size_t)s * 128 + g0) * n_heads + h;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 v = __ldg(src + (size_t)k * n_heads);
-      acc[k].x += wgt * v.x; acc[k].y += wgt * v.y; acc[k].z += wgt * v.z; acc[k].w += wgt * v.w;
-    }
+    const float4 v = __ldg(reinterpret_cast<const float4*>(o_part) + ((size_t)s * 128 + g) * n_heads + h);
+    acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
   }
-  uint4* dst = reinterpret_cast<uint4*>(o_lat + ((size_t)n * n_heads + h) * 512 + 4 * g0);
-  dst[0] = make_uint4(ptx::pack_bf16(acc[0].x, acc[0].y), ptx::pack_bf16(acc[0].z, acc[0].w),
-                      ptx::pack_bf16(acc[1].x, acc[1].y), ptx::pack_bf16(acc[1].z, acc[1].w));
-  dst[1] = make_uint4(ptx::pack_bf16(acc[2].x, acc[2].y), ptx::pack_bf16(acc[2].z, acc[2].w),
-                      ptx::pack_bf16(acc[3].x, acc[3].y), ptx::pack_bf16(acc[3].z, acc[3].w));
-  if (lse_out && blockIdx.y == 0 && half == 0)
+  *reinterpret_cast<uint2*>(o_lat + ((size_t)n * n_heads + h) * 512 + 4 * g) =
+      make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
+  if (lse_out && blockIdx.y == 0 && grp == 0)
     lse_out[(size_t)n * n_heads + h] = z > 0.f ? lmax + __logf(z) : -CUDART_INF_F;
 }
 

@@ -99,7 +99,9 @@ struct Bars {
   uint64_t x_sendok[2];  // peer has consumed its tile b, which this CTA may refill (8 remote arrivals)
   uint64_t p_full[2];    // P buffer b written (O rescaled if needed), 8 softmax warps
   uint64_t p_free[2];    // PV product that read P buffer b is complete
-  uint64_t o_full, o_free, qk_done, pv_done;
+  uint64_t o_full;        // PV product of a page complete (awaited one page behind, for rescaling)
+  uint64_t o_done;        // every PV product of the current item complete (epilogue)
+  uint64_t o_free, qk_done, pv_done;
   uint64_t pmax[2][4];   // the two softmax warps of row quarter q posted their page-b half-row maxima
   uint64_t lsum[4];      // the two softmax warps of row quarter q posted their half-row sums (per item)
 };
@@ -171,6 +173,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     }
     for (int b = 0; b < 2; ++b) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);   // armed for pages 0, 1
     mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, kSoftWarps);
     mbar_init(&bars->qk_done, 1);
     mbar_init(&bars->pv_done, 1);
@@ -310,6 +313,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           mma_commit(&bars->kv_empty[s]);
           mma_commit(&bars->o_full);
         }
+        // o_full alone cannot tell the last page's completion from the one before
+        // (a parity wait sees one phase at a time), so the epilogue waits on this
+        if (ok) mma_commit(&bars->o_done);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -531,8 +537,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 
       // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot
       {
-        const int gl = g + n - 1;
-        if (!warp_wait(&bars->o_full, gl & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait(&bars->o_done, ii & 1, abort_flag)) goto softmax_fail;
         tc_fence_after();
         float* ls = s_lsum + (ii & 1) * 2 * kRows;    // [item parity][half][row]
         ls[c * kRows + r] = l_run;

@@ -4,11 +4,15 @@
 // the s_q new tokens is its own row group (with s_q = 2 the two groups run
 // side by side on disjoint halves of the clusters and walk the same pages at
 // the same time, so the second read of a page tends to hit L2).  Within a
-// group the rows' pages are concatenated in sequence order and cut into
-// `clusters_per_group` contiguous ranges of equal size (floor(c * P / G));
-// the intersection of a range with a row is one work item.  A row that falls
-// inside a single range is written directly; a row cut by range boundaries
-// gets one partial slot per piece, numbered consecutively in row order.
+// group the rows are laid end to end in sequence order, each preceded by
+// kItemCostPages virtual pages that stand for the fixed cost of starting a
+// work item (loading the row's query, writing its output), and this line of
+// P' units is cut into `clusters_per_group` contiguous ranges of equal size
+// (floor(c * P' / G)).  The intersection of a range with a row's real pages
+// is one work item, so a cluster that crosses a row boundary takes fewer
+// pages.  A row that falls inside a single range is written directly; a row
+// cut by range boundaries gets one partial slot per piece, numbered
+// consecutively in row order.
 #include "plan_format.h"
 #include "mla_internal.h"
 
@@ -52,10 +56,10 @@ mla_status_t build_plan(const mla_dims_t& d, const int32_t* seq_lens, int32_t nu
   std::vector<int32_t> row_pieces(N, 0);
   for (int32_t g = 0; g < groups; ++g) {
     int64_t P = 0;
-    for (int32_t n : group_rows[g]) P += pages[n];
+    for (int32_t n : group_rows[g]) P += kItemCostPages + pages[n];
     int64_t off = 0;
     for (int32_t n : group_rows[g]) {
-      const int64_t r0 = off, r1 = off + pages[n];
+      const int64_t r0 = off + kItemCostPages, r1 = r0 + pages[n];
       off = r1;
       for (int32_t c = 0; c < per_group; ++c) {
         const int64_t lo = (int64_t)c * P / per_group, hi = (int64_t)(c + 1) * P / per_group;

@@ -9,6 +9,10 @@ namespace mla {
 constexpr int32_t kPlanMagic = 0x314C414D;  // "MLA1" little-endian
 constexpr int kPlanHeaderWords = 16;
 constexpr int kItemWords = 8;
+// Planner cost of starting a work item, in pages: loading the row's q_lat
+// into TMEM and writing its output take about as long as three pages of the
+// attention pipeline.
+constexpr int32_t kItemCostPages = 3;
 
 enum PlanHeader : int {
   kHdrMagic = 0,

@@ -45,6 +45,25 @@ def test_out_uv_matches_oracle(mla, N, H):
     assert rel_fro(got.float().cpu().numpy(), want) < 5e-3
 
 
+@pytest.mark.parametrize("N,H", [(37, 128), (300, 5), (600, 2)])
+def test_projections_write_only_their_rows(mla, N, H):
+    """Token tiles past N are clipped: rows after the output view keep their contents."""
+    w = W.make_workload(1, 1, H, [1], seed=N)
+    g = torch.Generator().manual_seed(N + 1)
+    q = torch.randn((N, H, 128), generator=g).to(torch.bfloat16).cuda()
+    o = (torch.randn((N, H, 512), generator=g) * 0.05).to(torch.bfloat16).cuda()
+    big_q = torch.full((N + 40, H, 512), 3.0, dtype=torch.bfloat16, device="cuda")
+    big_o = torch.full((N + 40, H, 128), 3.0, dtype=torch.bfloat16, device="cuda")
+    mla.absorb_q(q, w.w_uk.cuda(), big_q[:N])
+    mla.out_uv(o, w.w_uv.cuda(), big_o[:N])
+    torch.cuda.synchronize()
+    assert bool((big_q[N:] == 3.0).all()) and bool((big_o[N:] == 3.0).all())
+    want_q = O.contract(None, "absorb_q", "nhd,khd->nhk", q.cpu().double().numpy(), w.w_uk.double().numpy())
+    want_o = O.contract(None, "out_uv", "nhk,khv->nhv", o.cpu().double().numpy(), w.w_uv.double().numpy())
+    assert rel_fro(big_q[:N].float().cpu().numpy(), want_q) < 5e-3
+    assert rel_fro(big_o[:N].float().cpu().numpy(), want_o) < 5e-3
+
+
 # ------------------------------------------------------------------ page indexing
 def test_gather_pages_bit_exact(mla):
     w = W.make_workload(3, 1, 4, [130, 64, 5], seed=4, pool="scattered:2")
@@ -178,15 +197,17 @@ def test_full_size_preset_sampled(mla, name):
     _sampled(name)
 
 
-@pytest.mark.parametrize("name", ["long128k", "mtp2"])
+@pytest.mark.parametrize("name", ["v2_4k", "varlen", "long128k", "mtp2"])
 def test_full_size_bitwise_deterministic(mla, name):
-    """Repeated runs on the same inputs give identical bits (no race between
-    the cluster's score exchange, the softmax and the tensor-core pipeline)."""
+    """Repeated runs on the same inputs give identical bits, split partials
+    included (no race between the cluster's score exchange, the softmax, the
+    tensor-core pipeline and the epilogue)."""
     w = W.preset_workload(name)
     outs = []
     for _ in range(3):
-        _, res = run_gpu(w)
+        dec, res = run_gpu(w)
         assert res.status.item() == 0
-        outs.append((res.o_lat.clone(), res.out.clone(), res.lse.clone()))
+        outs.append((res.o_lat.clone(), res.out.clone(), res.lse.clone(), dec.o_part.clone(),
+                     dec.lse_part.clone()))
     for o in outs[1:]:
         assert all(torch.equal(a, b) for a, b in zip(outs[0], o))

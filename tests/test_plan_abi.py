@@ -23,10 +23,15 @@ def test_library_exports_every_declared_symbol():
 
 
 # ------------------------------------------------------------------ independent planner
+ITEM_COST_PAGES = 3
+
+
 def py_plan(seq_lens, s_q, causal, n_heads, num_clusters, page=64):
     """Re-derivation of the documented split rule: per query position i (its own
-    group of clusters when there are at least s_q clusters), the rows' pages are
-    concatenated in sequence order and cut at floor(c * P / G)."""
+    group of clusters when there are at least s_q clusters), the rows are laid
+    end to end in sequence order, each preceded by ITEM_COST_PAGES virtual
+    pages, and the line of P' units is cut at floor(c * P' / G); a piece is a
+    range's intersection with a row's real pages."""
     B = len(seq_lens)
     N = B * s_q
     rows = []
@@ -39,10 +44,11 @@ def py_plan(seq_lens, s_q, causal, n_heads, num_clusters, page=64):
     pieces = []   # (cluster, row, p0, p1)
     for g in range(groups):
         members = [n for n in range(N) if groups == 1 or n % s_q == g]
-        P = sum(rows[n]["pages"] for n in members)
+        P = sum(ITEM_COST_PAGES + rows[n]["pages"] for n in members)
         off = 0
         for n in members:
-            r0, r1 = off, off + rows[n]["pages"]
+            r0 = off + ITEM_COST_PAGES
+            r1 = r0 + rows[n]["pages"]
             off = r1
             for c in range(G):
                 lo, hi = c * P // G, (c + 1) * P // G
