@@ -31,6 +31,8 @@ __global__ void __launch_bounds__(kCombineThreads)
 mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o_part,
                    const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o_lat,
                    float* __restrict__ lse_out, int n_heads) {
+  ptx::griddep_wait();   // the attention kernel's partials are complete and visible
+  ptx::griddep_launch_dependents();
   const int n = blockIdx.x;
   const int h = threadIdx.x & 127;
   const int grp = threadIdx.x >> 7;
@@ -82,9 +84,9 @@ mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_
                             const float* o_part, const float* lse_part, void* o_lat,
                             float* lse_out, void* stream) {
   dim3 grid(n_rows, 512 / kCombineCols);
-  mla_combine_kernel<<<grid, kCombineThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      plan_dev, o_part, lse_part, static_cast<__nv_bfloat16*>(o_lat), lse_out, d.n_heads);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(mla_combine_kernel, grid, dim3(kCombineThreads), 0, stream, plan_dev, o_part, lse_part,
+                             static_cast<__nv_bfloat16*>(o_lat), lse_out, d.n_heads);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return MLA_OK;
 }

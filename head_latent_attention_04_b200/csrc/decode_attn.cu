@@ -146,14 +146,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   const int cid = (int)cluster_id_x();
 
   // The plan must match the launch (uniform over the grid).
-  const int32_t* plan = p.plan;
-  const bool plan_ok = plan[kHdrMagic] == kPlanMagic && plan[kHdrNumClusters] == p.num_clusters &&
-                       plan[kHdrNumRows] == p.n_rows && plan[kHdrHeads] == p.n_heads;
-  const int32_t* items = plan + plan[kHdrOffItems];
-  const int it_begin = plan_ok ? plan[plan[kHdrOffCluster] + cid] : 0;
-  const int it_end = plan_ok ? plan[plan[kHdrOffCluster] + cid + 1] : 0;
-  if (!plan_ok && threadIdx.x == 0 && rank == 0 && cid == 0) report(p.status, MLA_STATUS_BAD_SEQLEN);
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -197,43 +189,79 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   cluster_sync();   // peer barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();   // set-up above overlaps the previous kernel; global memory only from here
+  griddep_launch_dependents();
+
+  // The section offsets follow from the cluster count, so the cluster's item
+  // range is read without first waiting for the header (checked alongside).
+  const int32_t* plan = p.plan;
+  const int off_cluster = kPlanHeaderWords, off_items = kPlanHeaderWords + p.num_clusters + 1;
+  const int32_t* items = plan + off_items;
+  const int it_begin_raw = plan[off_cluster + cid], it_end_raw = plan[off_cluster + cid + 1];
+  const bool plan_ok = plan[kHdrMagic] == kPlanMagic && plan[kHdrNumClusters] == p.num_clusters &&
+                       plan[kHdrNumRows] == p.n_rows && plan[kHdrHeads] == p.n_heads &&
+                       plan[kHdrOffCluster] == off_cluster && plan[kHdrOffItems] == off_items;
+  const int it_begin = plan_ok ? it_begin_raw : 0;
+  const int it_end = plan_ok ? it_end_raw : 0;
+  if (!plan_ok && threadIdx.x == 0 && rank == 0 && cid == 0) report(p.status, MLA_STATUS_BAD_SEQLEN);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int g = 0;
-      for (int it = it_begin; it < it_end && !*abort_flag; ++it) {
-        const int32_t* w = items + (size_t)it * kItemWords;
-        const int b = w[kItB], row = w[kItRow];
-        const int ii = it - it_begin;
-        if (ii > 0 && !mbar_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto producer_fail;
-        mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
-        tma_load_3d(s_qrope, &tm_qrope, &bars->q_full, 32 * rank, 0, row);
-        if (it + 1 < it_end)   // the next item's q_lat rows, so that its loader reads them from L2
-          bulk_prefetch_l2(p.q_lat + (size_t)items[(size_t)(it + 1) * kItemWords + kItRow] * p.n_heads * 512,
-                           (uint32_t)p.n_heads * 1024u);
-        for (int pg = w[kItPageBegin]; pg < w[kItPageEnd]; ++pg, ++g) {
-          const int s = g % kStages;
-          if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, abort_flag))
-            goto producer_fail;
-          int blk = p.block_table[(size_t)b * p.max_blocks + pg];
-          if (blk < 0 || blk >= p.num_blocks) {
-            report(p.status, MLA_STATUS_BAD_BLOCK);
-            blk = 0;
-          }
-          uint8_t* st = s_kv + s * kStageBytes;
-          mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tma_load_2d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, blk * kPage);
-          tma_load_2d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, blk * kPage);
+    // Lane 0 waits and issues; the whole warp fetches block ids 32 pages at a
+    // time with one coalesced load, so a page's TMA never waits on its own
+    // block-table read.
+    int g = 0;
+    bool fail = false;
+    for (int it = it_begin; it < it_end && !fail && !*abort_flag; ++it) {
+      const int32_t* w = items + (size_t)it * kItemWords;
+      const int b = w[kItB], row = w[kItRow], pb = w[kItPageBegin], pe = w[kItPageEnd];
+      const int ii = it - it_begin;
+      if (lane == 0) {
+        if (ii > 0 && !mbar_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) {
+          fail = true;
+        } else {
+          mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
+          tma_load_3d(s_qrope, &tm_qrope, &bars->q_full, 32 * rank, 0, row);
+          if (it + 1 < it_end)   // the next item's q_lat rows, so that its loader reads them from L2
+            bulk_prefetch_l2(p.q_lat + (size_t)items[(size_t)(it + 1) * kItemWords + kItRow] * p.n_heads * 512,
+                             (uint32_t)p.n_heads * 1024u);
         }
       }
-      goto producer_drain;
-    producer_fail:
-      *abort_flag = 1;
-      report(p.status, MLA_STATUS_TIMEOUT);
-    producer_drain:
+      fail = __shfl_sync(0xffffffffu, fail, 0);
+      int my_blk = 0;
+      for (int pg = pb; pg < pe && !fail; ++pg, ++g) {
+        const int rel = pg - pb;
+        if ((rel & 31) == 0) {
+          const int q = pg + lane;
+          my_blk = q < pe ? p.block_table[(size_t)b * p.max_blocks + q] : 0;
+        }
+        int blk = __shfl_sync(0xffffffffu, my_blk, rel & 31);
+        if (lane == 0) {
+          const int s = g % kStages;
+          if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, abort_flag)) {
+            fail = true;
+          } else {
+            if (blk < 0 || blk >= p.num_blocks) {
+              report(p.status, MLA_STATUS_BAD_BLOCK);
+              blk = 0;
+            }
+            uint8_t* st = s_kv + s * kStageBytes;
+            mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tma_load_2d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, blk * kPage);
+            tma_load_2d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, blk * kPage);
+          }
+        }
+        fail = __shfl_sync(0xffffffffu, fail, 0);
+        if (fail) break;   // this page was not issued
+      }
+    }
+    if (lane == 0) {
+      if (fail) {
+        *abort_flag = 1;
+        report(p.status, MLA_STATUS_TIMEOUT);
+      }
       // every issued load must land before the CTA may exit
       for (int k = g - 1; k >= 0 && k >= g - kStages; --k)
         mbar_wait(&bars->kv_full[k % kStages], (k / kStages) & 1, nullptr);
@@ -547,6 +575,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         l_run = ls[r] + ls[kRows + r];             // same order in both halves
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const bool valid = r < p.n_heads;
+        const bool o_lat_32b = (reinterpret_cast<uintptr_t>(p.o_lat) & 31) == 0;
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
@@ -555,13 +584,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           if (!valid) continue;
           const int col = 256 * rank + 128 * c + 32 * q;
           if (slot < 0) {
-            uint4* dst = reinterpret_cast<uint4*>(p.o_lat + ((size_t)row * p.n_heads + r) * 512 + col);
+            uint32_t pk[16];
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(pack_bf16(__uint_as_float(o[8 * k]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
-                                  pack_bf16(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
-                                  pack_bf16(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
-                                  pack_bf16(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+            for (int k = 0; k < 16; ++k)
+              pk[k] = pack_bf16(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+            __nv_bfloat16* dst = p.o_lat + ((size_t)row * p.n_heads + r) * 512 + col;
+            if (o_lat_32b) {   // one full 32-byte sector per store
+              st_global_v8(dst, pk);
+              st_global_v8(dst + 16, pk + 8);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                reinterpret_cast<uint4*>(dst)[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+            }
           } else {
             // column-group-major partials: a warp's 32 rows of one 4-column group are contiguous
             float4* dst = reinterpret_cast<float4*>(p.o_part) + ((size_t)slot * 128 + col / 4) * p.n_heads + r;
@@ -649,8 +684,9 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
 
   cudaError_t e = decode_smem_attr();
   if (e == cudaSuccess) {
-    mla_decode_kernel<<<2 * num_clusters, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tm_kv, tm_rope, tm_q, p);
-    e = cudaGetLastError();
+    e = launch_pdl(mla_decode_kernel, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv, tm_rope,
+                   tm_q, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return MLA_OK;

@@ -108,6 +108,8 @@ absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();   // set-up above overlaps the previous kernel; global memory only from here
+  griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     mbar_arrive_expect_tx(full, 2 * kATileBytes + 2 * bn * 128);
@@ -180,6 +182,8 @@ out_uv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp == 0 && lane == 0) {
     for (int kc = 0; kc < kChunks; ++kc) {
@@ -279,8 +283,8 @@ mla_status_t launch_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, 
   GemmParams p{n_tokens, n_heads, bn, 0};
   cudaError_t e = set_smem_attrs();
   if (e == cudaSuccess) {
-    absorb_q_kernel<<<dim3(512 / kBM, n_heads, tiles), 128, smem, static_cast<cudaStream_t>(stream)>>>(tw, tx, to, p);
-    e = cudaGetLastError();
+    e = launch_pdl(absorb_q_kernel, dim3(512 / kBM, n_heads, tiles), dim3(128), smem, stream, tw, tx, to, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "absorb_q launch: %s", cudaGetErrorString(e));
   return MLA_OK;
@@ -302,8 +306,8 @@ mla_status_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int n
   GemmParams p{n_tokens, n_heads, bn, stages};
   cudaError_t e = set_smem_attrs();
   if (e == cudaSuccess) {
-    out_uv_kernel<<<dim3(1, n_heads, tiles), 128, smem, static_cast<cudaStream_t>(stream)>>>(tw, tx, to, p);
-    e = cudaGetLastError();
+    e = launch_pdl(out_uv_kernel, dim3(1, n_heads, tiles), dim3(128), smem, stream, tw, tx, to, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "out_uv launch: %s", cudaGetErrorString(e));
   return MLA_OK;

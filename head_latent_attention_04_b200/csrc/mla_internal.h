@@ -2,10 +2,32 @@
 #pragma once
 #include "../../include/mla.h"
 
+#include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace mla {
+
+// Launches `kernel` with programmatic stream serialization: it may begin its
+// set-up while the previous kernel in the stream is still running (every
+// kernel of the library calls ptx::griddep_wait() before touching global memory).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, void* stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Records a printf-style message in the thread-local error slot; returns `code`.
 mla_status_t set_error(mla_status_t code, const char* fmt, ...);

@@ -113,6 +113,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it in the stream still runs.  It must not touch global memory
+// before griddep_wait(), which returns once that kernel has completed and its
+// writes are visible.  griddep_launch_dependents() lets the next such kernel
+// start its own set-up early.  Both are no-ops without the launch attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -150,6 +161,13 @@ __device__ __forceinline__ void st_cluster_v4u(uint32_t cluster_addr, uint32_t a
                                                uint32_t d) {
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a), "r"(b),
                "r"(c), "r"(d)
+               : "memory");
+}
+
+// 32-byte global store of eight words (address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* gptr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(gptr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                : "memory");
 }
 

@@ -64,6 +64,29 @@ def test_projections_write_only_their_rows(mla, N, H):
     assert rel_fro(big_o[:N].float().cpu().numpy(), want_o) < 5e-3
 
 
+def test_kernels_wait_for_a_preceding_copy(mla):
+    """Every kernel may start early behind a preceding kernel, but a preceding
+    host-to-device copy on the stream still completes first: a large copy into
+    q_nope right before mla_absorb_q must be fully visible to it."""
+    H, N = 128, 256
+    w = W.make_workload(1, 1, H, [1], seed=3)
+    g = torch.Generator().manual_seed(5)
+    q_host = torch.randn((N, H, 128), generator=g).to(torch.bfloat16).pin_memory()
+    big = torch.empty(64 << 20, dtype=torch.uint8).pin_memory()          # keeps the copy engine busy first
+    big_dev = torch.empty_like(big, device="cuda")
+    q_dev = torch.zeros((N, H, 128), dtype=torch.bfloat16, device="cuda")
+    w_uk = w.w_uk.cuda()
+    out = torch.empty((N, H, 512), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    big_dev.copy_(big, non_blocking=True)
+    q_dev.copy_(q_host, non_blocking=True)
+    mla.absorb_q(q_dev, w_uk, out)
+    torch.cuda.synchronize()
+    want = mla.absorb_q(q_host.cuda(), w_uk)
+    torch.cuda.synchronize()
+    assert torch.equal(out, want)
+
+
 # ------------------------------------------------------------------ page indexing
 def test_gather_pages_bit_exact(mla):
     w = W.make_workload(3, 1, 4, [130, 64, 5], seed=4, pool="scattered:2")
