@@ -15,8 +15,9 @@ a 256 MB buffer (outside the events); the K-step region is bracketed by a
 barrier and torch.cuda.synchronize() on both sides; ms_per_step is the mean
 per-step event time, max over ranks.  The attention kernel alone is timed the
 same way for the roofline.  `e2e` repeats the step through the public
-Decoder API with the step's inputs (queries, page table) copied from pinned
-host memory and the output copied back, inside the timed region.
+mla.GraphedStep API: the step's inputs (queries, page table) copied from
+pinned host memory, the kernels, and the output copied back to pinned host
+memory, all inside the timed region.
 
 Multi-GPU (torchrun, one process per GPU): data-parallel replicas.  Each rank
 decodes its own batch of the same shape (weak scaling); no collective runs on
@@ -323,31 +324,54 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ms_local = statistics.fmean(step_ms)
     attn_local = statistics.fmean(attn_ms)
 
-    # e2e: the public API with host buffers (queries + page table in, output out)
-    qn_h = w.q_nope.cpu().pin_memory()
-    qr_h = w.q_rope.cpu().pin_memory()
-    bt_h = torch.as_tensor(w.block_table).pin_memory()
-    out_h = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
-    qn_d, qr_d, bt_d = torch.empty_like(w.q_nope), torch.empty_like(w.q_rope), torch.empty_like(bt)
-    h2d = qn_h.numel() * 2 + qr_h.numel() * 2 + bt_h.numel() * 4
-    d2h = out_h.numel() * 2
+    # e2e, from host buffers to host buffers through the public API.
+    # Serial (latency): mla.GraphedStep replays one graph per step (pinned H2D of
+    # the queries and page table, the four kernels, D2H of the output), with L2
+    # flushed before every step outside the events.
+    gs = mla.GraphedStep(dec, w.kv_pool, w.w_uk, w.w_uv)
+    gs.q_nope.copy_(w.q_nope.cpu())
+    gs.q_rope.copy_(w.q_rope.cpu())
+    gs.block_table.copy_(torch.as_tensor(w.block_table))
+    h2d, d2h = gs.h2d_bytes, gs.d2h_bytes
+    for _ in range(args.warmup):
+        gs.run(sync=False)
     ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     barrier()
     for i in range(K):
         flush.zero_()
         ee[i][0].record(stream)
-        qn_d.copy_(qn_h, non_blocking=True)
-        qr_d.copy_(qr_h, non_blocking=True)
-        bt_d.copy_(bt_h, non_blocking=True)
-        r = dec.run(qn_d, qr_d, w.kv_pool, bt_d, w.w_uk, w.w_uv)
-        out_h.copy_(r.out, non_blocking=True)
+        gs.run(sync=False)
         ee[i][1].record(stream)
     barrier()
-    e2e_local = statistics.fmean(a.elapsed_time(b) for a, b in ee)
+    serial_ms = statistics.fmean(a.elapsed_time(b) for a, b in ee)
+    e2e_check = bool(torch.equal(gs.out, dec.out.cpu()))
+    del gs
+    # Streamed (throughput): mla.StreamedDecoder overlaps each step's copies with
+    # its neighbours' kernels; K back-to-back steps timed as one region.  No
+    # flush inside the region: every step streams the whole KV cache, which is
+    # larger than L2 for the full-size workloads.
+    sd = mla.StreamedDecoder(dec, w.kv_pool, w.w_uk, w.w_uv)
+    for qn_h, qr_h, bt_h in sd.host_in:
+        qn_h.copy_(w.q_nope.cpu())
+        qr_h.copy_(w.q_rope.cpu())
+        bt_h.copy_(torch.as_tensor(w.block_table))
+    for _ in range(args.warmup):
+        sd.submit()
+    barrier()
+    s_in, _, s_out = sd.streams
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for _ in range(K):
+        last = sd.submit()
+    e1.record(s_out)
+    barrier()
+    e2e_local = e0.elapsed_time(e1) / K
+    e2e_check = e2e_check and bool(torch.equal(sd.wait(last), dec.out.cpu()))
+    del sd
     status = int(dec.status.item())
 
     # bookkeeping collectives only (identity at one rank): max over ranks, status OR
-    ms, attn, e2e = dp.reduce_max([ms_local, attn_local, e2e_local], device=dev)
+    ms, attn, e2e, serial_ms = dp.reduce_max([ms_local, attn_local, e2e_local, serial_ms], device=dev)
     status = dp.reduce_status(status, device=dev)
     used_graph = graph is not None
     del graph
@@ -382,7 +406,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "step_roofline_frac": step_roof_s / (ms * 1e-3),
         "roofline": roof,
         "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
+                "path": "mla.StreamedDecoder: pinned H2D and D2H of each step overlapped with the "
+                        "neighbouring steps' kernels, K steps timed as one region (KV cache > L2, no flush)",
+                "serial_ms_per_step": serial_ms,
+                "serial_path": "mla.GraphedStep: H2D, 4 kernels, D2H in one graph per step, L2 flushed "
+                               "before each step",
+                "matches_device_output": e2e_check},
         "gpu_launches": K * dec.launches_per_step + K,
         "clocks": sampler.summary(),
         "device_status": status,

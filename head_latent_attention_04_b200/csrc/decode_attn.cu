@@ -590,8 +590,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
               pk[k] = pack_bf16(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
             __nv_bfloat16* dst = p.o_lat + ((size_t)row * p.n_heads + r) * 512 + col;
             if (o_lat_32b) {   // one full 32-byte sector per store
-              st_global_v8(dst, pk);
-              st_global_v8(dst + 16, pk + 8);
+              st_global_v8(dst, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+              st_global_v8(dst + 16, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14], pk[15]);
             } else {
 #pragma unroll
               for (int k = 0; k < 4; ++k)

@@ -230,6 +230,151 @@ class Decoder:
         return 4 if self.num_slots > 0 else 3
 
 
+class GraphedStep:
+    """One decode step from host memory to host memory, replayed as a CUDA graph.
+
+    For a serving loop with a fixed batch shape: the step's inputs live in
+    pinned host buffers (``q_nope``, ``q_rope``, ``block_table``); ``run()``
+    replays one graph that copies them to the device, runs absorb ->
+    attention -> combine -> out_uv, and copies ``out`` back to the pinned
+    ``out`` buffer.  The graph fixes every pointer, so the cache pool, the
+    weights and the decoder's buffers must outlive this object; refill the
+    host buffers in place between calls.
+    """
+
+    def __init__(self, decoder: Decoder, kv_pool, w_uk, w_uv, stream=None):
+        dev = kv_pool.device
+        N, H = decoder.N, decoder.H
+        self.decoder = decoder
+        self.q_nope = torch.zeros((N, H, 128), dtype=torch.bfloat16).pin_memory()
+        self.q_rope = torch.zeros((N, H, 64), dtype=torch.bfloat16).pin_memory()
+        self.block_table = torch.zeros((decoder.B, decoder.dims.max_blocks_per_seq), dtype=torch.int32).pin_memory()
+        self.out = torch.empty((N, H, 128), dtype=torch.bfloat16).pin_memory()
+        self._q_nope = torch.empty(self.q_nope.shape, dtype=torch.bfloat16, device=dev)
+        self._q_rope = torch.empty(self.q_rope.shape, dtype=torch.bfloat16, device=dev)
+        self._bt = torch.empty(self.block_table.shape, dtype=torch.int32, device=dev)
+        self._args = (kv_pool, w_uk, w_uv)
+        self.graph = torch.cuda.CUDAGraph()
+        s = stream or torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            self._body()                      # warm-up outside capture (lazy library set-up)
+            torch.cuda.synchronize(dev)
+            with torch.cuda.graph(self.graph, stream=s):
+                self._body()
+        torch.cuda.synchronize(dev)
+
+    def _body(self):
+        kv_pool, w_uk, w_uv = self._args
+        self._q_nope.copy_(self.q_nope, non_blocking=True)
+        self._q_rope.copy_(self.q_rope, non_blocking=True)
+        self._bt.copy_(self.block_table, non_blocking=True)
+        r = self.decoder.run(self._q_nope, self._q_rope, kv_pool, self._bt, w_uk, w_uv)
+        self.out.copy_(r.out, non_blocking=True)
+
+    def run(self, sync: bool = True) -> torch.Tensor:
+        """Replays the step on the current stream; returns the pinned ``out`` buffer."""
+        self.graph.replay()
+        if sync:
+            torch.cuda.current_stream().synchronize()
+        return self.out
+
+    @property
+    def h2d_bytes(self) -> int:
+        return self.q_nope.nbytes + self.q_rope.nbytes + self.block_table.nbytes
+
+    @property
+    def d2h_bytes(self) -> int:
+        return self.out.nbytes
+
+
+class StreamedDecoder:
+    """Back-to-back decode steps from pinned host memory to pinned host memory,
+    with the copies of one step overlapping the kernels of its neighbours.
+
+    ``depth`` input/output sets rotate: step k uses set i = k % depth.  The user
+    fills ``host_in[i]`` (q_nope, q_rope, block_table), calls ``submit()``, and
+    reads ``host_out[i]`` once ``ready(i)`` (or ``wait(i)``) says the step's
+    device-to-host copy is done.  Three streams carry the work: host-to-device
+    copies, the kernels (one CUDA graph per set: absorb -> attention ->
+    combine -> out_uv, then a device copy of the output into the set's
+    buffer), and device-to-host copies; events keep each set's buffers from
+    being overwritten while still in use.  The decoder's scratch buffers are
+    shared, so the kernels of consecutive steps run one after another.
+    """
+
+    def __init__(self, decoder: Decoder, kv_pool, w_uk, w_uv, depth: int = 2):
+        dev = kv_pool.device
+        N, H, B = decoder.N, decoder.H, decoder.B
+        mb = decoder.dims.max_blocks_per_seq
+        self.depth = depth
+        self.host_in = [(torch.zeros((N, H, 128), dtype=torch.bfloat16).pin_memory(),
+                         torch.zeros((N, H, 64), dtype=torch.bfloat16).pin_memory(),
+                         torch.zeros((B, mb), dtype=torch.int32).pin_memory()) for _ in range(depth)]
+        self.host_out = [torch.empty((N, H, 128), dtype=torch.bfloat16).pin_memory() for _ in range(depth)]
+        self._dev_in = [(torch.empty((N, H, 128), dtype=torch.bfloat16, device=dev),
+                         torch.empty((N, H, 64), dtype=torch.bfloat16, device=dev),
+                         torch.empty((B, mb), dtype=torch.int32, device=dev)) for _ in range(depth)]
+        self._dev_out = [torch.empty((N, H, 128), dtype=torch.bfloat16, device=dev) for _ in range(depth)]
+        self._s_in, self._s_cmp, self._s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+        self._ev_in = [torch.cuda.Event() for _ in range(depth)]
+        self._ev_cmp = [torch.cuda.Event() for _ in range(depth)]
+        self._ev_out = [torch.cuda.Event() for _ in range(depth)]
+        self._graphs = []
+        self._s_cmp.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(self._s_cmp):
+            for i in range(depth):
+                qn, qr, bt = self._dev_in[i]
+                qn.zero_(); qr.zero_(); bt.zero_()
+                decoder.run(qn, qr, kv_pool, bt, w_uk, w_uv)   # warm-up outside capture
+                torch.cuda.synchronize(dev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=self._s_cmp):
+                    r = decoder.run(qn, qr, kv_pool, bt, w_uk, w_uv)
+                    self._dev_out[i].copy_(r.out)
+                self._graphs.append(g)
+        torch.cuda.synchronize(dev)
+        self.steps = 0
+
+    def submit(self) -> int:
+        """Enqueues the next step on the next set; returns the set index."""
+        i = self.steps % self.depth
+        reuse = self.steps >= self.depth
+        if reuse:   # this set's device inputs are free once its previous step's kernels finished
+            self._s_in.wait_event(self._ev_cmp[i])
+        with torch.cuda.stream(self._s_in):
+            for d, h in zip(self._dev_in[i], self.host_in[i]):
+                d.copy_(h, non_blocking=True)
+            self._ev_in[i].record(self._s_in)
+        self._s_cmp.wait_event(self._ev_in[i])
+        if reuse:   # and its device output once its previous copy back finished
+            self._s_cmp.wait_event(self._ev_out[i])
+        with torch.cuda.stream(self._s_cmp):
+            self._graphs[i].replay()
+            self._ev_cmp[i].record(self._s_cmp)
+        self._s_out.wait_event(self._ev_cmp[i])
+        with torch.cuda.stream(self._s_out):
+            self.host_out[i].copy_(self._dev_out[i], non_blocking=True)
+            self._ev_out[i].record(self._s_out)
+        self.steps += 1
+        return i
+
+    def input_free(self, i: int) -> bool:
+        """``host_in[i]`` may be refilled once its last host-to-device copy is done."""
+        return self._ev_in[i].query()
+
+    def ready(self, i: int) -> bool:
+        return self._ev_out[i].query()
+
+    def wait(self, i: int) -> torch.Tensor:
+        self._ev_out[i].synchronize()
+        return self.host_out[i]
+
+    @property
+    def streams(self):
+        return self._s_in, self._s_cmp, self._s_out
+
+
 def decode(q_nope, q_rope, kv_pool, block_table, seq_lens, w_uk, w_uv, s_q=1, scale=None,
            causal=True, num_clusters=None) -> DecodeOutputs:
     """One-shot absorbed MLA decode on device tensors (see ``Decoder``)."""

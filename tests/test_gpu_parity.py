@@ -87,6 +87,61 @@ def test_kernels_wait_for_a_preceding_copy(mla):
     assert torch.equal(out, want)
 
 
+def test_graphed_step_host_to_host(mla):
+    """mla.GraphedStep (pinned H2D, the four kernels, D2H in one CUDA graph)
+    gives the Decoder's output, and follows new host inputs on each replay."""
+    w = W.make_workload(3, 2, 64, [300, 5, 1000], seed=21, pool="scattered:1.5")
+    dev = torch.device("cuda")
+    wd = w.to(dev)
+    dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev)
+    gs = mla.GraphedStep(dec, wd.kv_pool, wd.w_uk, wd.w_uv)
+    g = torch.Generator().manual_seed(9)
+    for _ in range(2):
+        q_nope = torch.randn(w.q_nope.shape, generator=g).to(torch.bfloat16)
+        q_rope = torch.randn(w.q_rope.shape, generator=g).to(torch.bfloat16)
+        gs.q_nope.copy_(q_nope)
+        gs.q_rope.copy_(q_rope)
+        gs.block_table.copy_(torch.as_tensor(w.block_table))
+        got = gs.run().clone()
+        ref = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev).run(
+            q_nope.to(dev), q_rope.to(dev), wd.kv_pool, torch.as_tensor(w.block_table, device=dev), wd.w_uk, wd.w_uv)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref.out.cpu())
+    assert gs.h2d_bytes == w.q_nope.nbytes + w.q_rope.nbytes + w.block_table.size * 4
+    assert dec.status.item() == 0
+
+
+def test_streamed_decoder_overlapped_steps(mla):
+    """mla.StreamedDecoder: steps with different inputs in flight at once each
+    return the output the Decoder gives for their own inputs."""
+    w = W.make_workload(4, 1, 32, [700, 64, 65, 2000], seed=31)
+    dev = torch.device("cuda")
+    wd = w.to(dev)
+    bt = torch.as_tensor(w.block_table, device=dev)
+    dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev)
+    sd = mla.StreamedDecoder(dec, wd.kv_pool, wd.w_uk, wd.w_uv, depth=2)
+    g = torch.Generator().manual_seed(2)
+    inputs, sets = [], []
+    for k in range(5):
+        i = k % 2
+        while not sd.input_free(i):
+            pass
+        if k >= 2:
+            sd.wait(i)   # the previous output of this set was checked below
+        qn = torch.randn(w.q_nope.shape, generator=g).to(torch.bfloat16)
+        qr = torch.randn(w.q_rope.shape, generator=g).to(torch.bfloat16)
+        sd.host_in[i][0].copy_(qn)
+        sd.host_in[i][1].copy_(qr)
+        sd.host_in[i][2].copy_(torch.as_tensor(w.block_table))
+        assert sd.submit() == i
+        got = sd.wait(i).clone()
+        ref = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev).run(
+            qn.to(dev), qr.to(dev), wd.kv_pool, bt, wd.w_uk, wd.w_uv)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref.out.cpu())
+    assert dec.status.item() == 0
+
+
 # ------------------------------------------------------------------ page indexing
 def test_gather_pages_bit_exact(mla):
     w = W.make_workload(3, 1, 4, [130, 64, 5], seed=4, pool="scattered:2")
