@@ -201,6 +201,52 @@ def cpu_oracle_sample(w, seconds: float, max_rows: int | None = None):
     return done / el, done, el, cores
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_absorbed_fp32(w, b: int, w_uk=None, w_uv=None):
+    """The absorbed order (order 2 of "MLA Matrix Absorption Analysis", sections
+    2.2 and 3.2) for sequence b in float32 NumPy with BLAS: returns out [s][h][128]."""
+    w_uk = w.w_uk.cpu().float().numpy() if w_uk is None else w_uk   # [512][h][128]
+    w_uv = w.w_uv.cpu().float().numpy() if w_uv is None else w_uv
+    rows = slice(b * w.s_q, (b + 1) * w.s_q)
+    qn = w.q_nope[rows].cpu().float().numpy()       # [s][h][128]
+    qr = w.q_rope[rows].cpu().float().numpy()       # [s][h][64]
+    cache = w.cache_rows(b).cpu().float().numpy()
+    ckv, kr = cache[:, :512], cache[:, 512:]
+    T = cache.shape[0]
+    q_lat = np.einsum("shd,khd->shk", qn, w_uk, optimize=True)
+    sc = (q_lat @ ckv.T + qr @ kr.T) * np.float32(1.0 / math.sqrt(192.0))   # [s][h][T]
+    for i in range(w.s_q):
+        sc[i, :, T - w.s_q + 1 + i:] = -np.inf
+    sc -= sc.max(-1, keepdims=True)
+    p = np.exp(sc)
+    p /= p.sum(-1, keepdims=True)
+    return np.einsum("shk,khv->shv", p @ ckv, w_uv, optimize=True)
+
+
+def cpu_absorbed_fp32_sample(w, seconds: float):
+    """A fairer CPU number beside the oracle: cpu_absorbed_fp32 on whole
+    sequences until `seconds`; returns (rows/s, rows, seconds)."""
+    w_uk = w.w_uk.cpu().float().numpy()
+    w_uv = w.w_uv.cpu().float().numpy()
+    done, t0 = 0, time.perf_counter()
+    for b in range(w.B):
+        cpu_absorbed_fp32(w, b, w_uk, w_uv)
+        done += w.s_q
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    return done / el, done, el
+
+
 # ----------------------------------------------------------------------------- arms
 def run_reference(args, rank: int, world: int):
     if rank != 0:
@@ -323,6 +369,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     attn_ms = [a.elapsed_time(b) for a, b in ea]
     ms_local = statistics.fmean(step_ms)
     attn_local = statistics.fmean(attn_ms)
+    pct = lambda xs: {"p10": float(np.percentile(xs, 10)), "p50": float(np.percentile(xs, 50)),
+                      "p90": float(np.percentile(xs, 90))}
+    step_pct, attn_pct = pct(step_ms), pct(attn_ms)
 
     # e2e, from host buffers to host buffers through the public API.
     # Serial (latency): mla.GraphedStep replays one graph per step (pinned H2D of
@@ -404,6 +453,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "attn_cache_tbs": acc["cache_bytes"] / (attn * 1e-3) / 1e12,
         "tflops": acc["step_flops"] * world / (ms * 1e-3) / 1e12,
         "step_roofline_frac": step_roof_s / (ms * 1e-3),
+        "ms_per_step_percentiles": step_pct,
+        "attention_ms_percentiles": attn_pct,
         "roofline": roof,
         "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
@@ -421,8 +472,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world == 1 and not args.no_cpu_baseline:
         rate, rows, secs, cores = cpu_oracle_sample(w, args.cpu_seconds)
         res["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                               "cpu_model": cpu_model(),
                                "sample": f"{rows} query rows of {args.config} (all heads, full context), "
                                          f"{secs:.1f} s, float64 order-1 oracle"}
+        rate32, rows32, secs32 = cpu_absorbed_fp32_sample(w, args.cpu_seconds / 3)
+        res["cpu_absorbed_fp32"] = {"value": rate32, "unit": "tokens/s", "cores": cores,
+                                    "sample": f"{rows32} query rows of {args.config}, {secs32:.1f} s, "
+                                              "float32 NumPy order 2 (a fairer CPU figure, not a target)"}
     return res
 
 

@@ -1,0 +1,29 @@
+"""CPU pieces of bench.py: the fairer float32 absorbed-order CPU figure computes
+the same attention as the oracle, and the algorithmic accounting matches the
+formulas the measurement uses."""
+import numpy as np
+
+import bench
+from head_latent_attention_04_b200 import workloads as W
+from oracle import mla_oracle as O
+
+
+def test_cpu_absorbed_fp32_matches_oracle():
+    w = W.make_workload(3, 2, 8, [5, 70, 130], seed=4)
+    for b in range(w.B):
+        rows = slice(b * w.s_q, (b + 1) * w.s_q)
+        ref = O.mla_decode(w.q_nope[rows].double().numpy(), w.q_rope[rows].double().numpy(),
+                           [w.cache_rows(b).double().numpy()], w.w_uk.double().numpy(),
+                           w.w_uv.double().numpy(), w.s_q, with_intermediates=False)["out"]
+        got = bench.cpu_absorbed_fp32(w, b)
+        np.testing.assert_allclose(got, ref, rtol=2e-4, atol=2e-5)
+
+
+def test_algorithmic_accounting():
+    acc = bench.algorithmic([4096] * 32, 1, 128)
+    assert acc["cache_bytes"] == 32 * 4096 * 1152
+    assert acc["attn_flops"] == 32 * 4096 * 2 * 128 * (2 * 512 + 64)
+    assert acc["attn_bytes"] == 32 * 4096 * 1152 + 32 * 128 * (576 + 512) * 2
+    # causal MTP: query i of a sequence of length T attends T - 1 + i keys
+    acc2 = bench.algorithmic([10, 20], 2, 128)
+    assert acc2["attn_flops"] == (9 + 10 + 19 + 20) * 2 * 128 * (2 * 512 + 64)
