@@ -76,7 +76,7 @@ static mla_status_t check_dims(const mla_dims_t* d) {
   if (d->d_nope != 128 || d->d_rope != 64 || d->d_c != 512 || d->d_v != 128 || d->page_size != 64)
     return set_error(MLA_ERR_UNSUPPORTED,
                      "only d_nope=128, d_rope=64, d_c=512, d_v=128, page_size=64 are supported");
-  if (d->s_q != 1 && d->s_q != 2) return set_error(MLA_ERR_UNSUPPORTED, "s_q must be 1 or 2");
+  if (d->s_q < 1 || d->s_q > 8) return set_error(MLA_ERR_UNSUPPORTED, "s_q must be in [1, 8]");
   if (d->n_heads < 1 || d->n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
   if (!(d->scale > 0.f) || d->scale != d->scale) return set_error(MLA_ERR_INVALID_ARG, "scale must be > 0");
   if ((int64_t)d->num_blocks * 64 > INT32_MAX) return set_error(MLA_ERR_UNSUPPORTED, "pool too large");

@@ -1,9 +1,9 @@
 // Host split-KV planner for the persistent decode kernel.
 //
 // Work unit: one page (64 keys) of one query row.  Each query position i of
-// the s_q new tokens is its own row group (with s_q = 2 the two groups run
-// side by side on disjoint halves of the clusters and walk the same pages at
-// the same time, so the second read of a page tends to hit L2).  Within a
+// the s_q new tokens is its own row group (the s_q groups run side by side on
+// disjoint sets of clusters and walk the same pages at about the same time,
+// so the repeated reads of a page tend to hit L2).  Within a
 // group the rows are laid end to end in sequence order, each preceded by
 // kItemCostPages virtual pages that stand for the fixed cost of starting a
 // work item (loading the row's query, writing its output), and this line of

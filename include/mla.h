@@ -34,7 +34,7 @@
  *
  * Shapes: n_tokens N = B * s_q query rows; row n = b * s_q + i.
  * Supported: d_nope = 128, d_rope = 64, d_c = 512, d_v = 128, page_size = 64,
- * s_q in {1, 2}, 1 <= n_heads <= 128.  Other shapes return MLA_ERR_UNSUPPORTED.
+ * 1 <= s_q <= 8, 1 <= n_heads <= 128.  Other shapes return MLA_ERR_UNSUPPORTED.
  */
 #ifndef MLA_H_
 #define MLA_H_
@@ -63,7 +63,7 @@ typedef enum {
 /* Problem dimensions of one decode batch. */
 typedef struct {
   int32_t B;                  /* sequences */
-  int32_t s_q;                /* new query tokens per sequence (1, or 2 for MTP) */
+  int32_t s_q;                /* new query tokens per sequence: 1, or up to 8 speculative (MTP) */
   int32_t n_heads;            /* h */
   int32_t d_nope;             /* 128 */
   int32_t d_rope;             /* 64 */
@@ -73,7 +73,7 @@ typedef struct {
   int32_t max_blocks_per_seq; /* columns of block_table */
   int32_t num_blocks;         /* blocks in the cache pool */
   float scale;                /* softmax scale, e.g. 1/sqrt(d_nope + d_rope) */
-  int32_t causal;             /* s_q == 2: 1 = query i attends t <= T - s_q + i; 0 = all T */
+  int32_t causal;             /* s_q > 1: 1 = query i attends t <= T - s_q + i; 0 = all T */
 } mla_dims_t;
 
 /* Library version (major * 10000 + minor * 100 + patch). */

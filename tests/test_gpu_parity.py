@@ -213,6 +213,15 @@ def test_mtp_causal(mla, lens, clusters):
     _full_check(w, num_clusters=clusters)
 
 
+@pytest.mark.parametrize("s_q,lens,clusters", [(3, [3, 64, 65, 1000, 130], 74), (4, [4, 200, 4100], 7),
+                                                (8, [8, 9, 70, 640], 74), (3, [5, 3000], 1)])
+def test_speculative_causal(mla, s_q, lens, clusters):
+    """s_q up to 8 new tokens per sequence (longer speculative queries), causal
+    among them: query i attends keys t <= T - s_q + i."""
+    w = W.make_workload(len(lens), s_q, 128, lens, seed=s_q * 7 + clusters, pool="permuted")
+    _full_check(w, num_clusters=clusters)
+
+
 def test_pool_permutation_is_bit_exact(mla):
     """Same values, different page placement, same plan -> identical bits."""
     a = W.make_workload(4, 1, 128, [300, 1000, 64, 513], seed=21, pool="contiguous")

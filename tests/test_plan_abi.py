@@ -93,6 +93,9 @@ def _unpack(buf):
     dict(lens=[2, 3, 64, 65, 66, 4097, 130], s_q=2, H=128, C=74),
     dict(lens=[2, 3, 64, 65, 66, 4097, 130], s_q=2, H=128, C=1),
     dict(lens=[77, 9000, 300], s_q=2, H=64, C=7),
+    dict(lens=[3, 64, 65, 5000, 130], s_q=3, H=128, C=74),
+    dict(lens=[8, 9, 700, 64], s_q=8, H=16, C=5),
+    dict(lens=[4, 4100], s_q=4, H=128, C=3),
     dict(lens=[100], s_q=1, H=1, C=3),
 ])
 def test_plan_bit_exact(case):
@@ -110,7 +113,7 @@ def test_plan_bit_exact(case):
 def test_plan_random_covers_every_page_once(seed):
     rng = np.random.default_rng(seed)
     B = int(rng.integers(1, 40))
-    s_q = int(rng.integers(1, 3))
+    s_q = int(rng.integers(1, 9))
     lens = rng.integers(s_q, 20000, size=B).tolist()
     C = int(rng.integers(1, 200))
     dims = mla.make_dims(B, s_q, 128, max(-(-t // 64) for t in lens), 10 ** 6)
@@ -135,7 +138,8 @@ def test_plan_random_covers_every_page_once(seed):
 # ------------------------------------------------------------------ validation (no GPU needed)
 def test_invalid_arguments_return_codes():
     good = mla.make_dims(2, 1, 16, 4, 8)
-    for field, val, code in [("d_c", 256, mla.MLA_ERR_UNSUPPORTED), ("s_q", 3, mla.MLA_ERR_UNSUPPORTED),
+    for field, val, code in [("d_c", 256, mla.MLA_ERR_UNSUPPORTED), ("s_q", 9, mla.MLA_ERR_UNSUPPORTED),
+                             ("s_q", 0, mla.MLA_ERR_UNSUPPORTED),
                              ("n_heads", 129, mla.MLA_ERR_UNSUPPORTED), ("page_size", 32, mla.MLA_ERR_UNSUPPORTED),
                              ("B", 0, mla.MLA_ERR_INVALID_ARG), ("scale", -1.0, mla.MLA_ERR_INVALID_ARG)]:
         d = mla.make_dims(2, 1, 16, 4, 8)
