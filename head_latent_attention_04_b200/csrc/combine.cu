@@ -13,7 +13,7 @@
 // HBM-bound: a block takes one row and 16 columns; thread (h, group) reads one
 // 4-column group of every piece (consecutive h -> coalesced 16-byte loads) and
 // writes 4 bf16 of its head.  Small grids (few rows cut into many pieces) still
-// get N x 32 blocks, and each thread's loads over the pieces are independent.
+// get N x 32 blocks; the pieces are merged in one pass, four at a time.
 #include "mla_internal.h"
 #include "plan_format.h"
 #include "ptx.cuh"
@@ -41,28 +41,40 @@ mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o
   const int s0 = rs[n], s1 = rs[n + 1];
   if (s1 <= s0) return;   // row written whole by the attention kernel
 
-  float lmax = -CUDART_INF_F;
-  for (int s = s0; s < s1; ++s) lmax = fmaxf(lmax, __ldg(lse_part + (size_t)s * n_heads + h));
-  float z = 0.f;
-  for (int s = s0; s < s1; ++s) {
-    const float l = __ldg(lse_part + (size_t)s * n_heads + h);
-    z += (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax);
+  // One pass over the pieces, four at a time with all their loads in flight,
+  // keeping a running maximum of the LSEs and rescaling the sums when it grows.
+  const int g = blockIdx.y * (kCombineCols / 4) + grp;   // this thread's 4-column group
+  const float4* src = reinterpret_cast<const float4*>(o_part) + (size_t)g * n_heads + h;
+  const size_t slot_stride = (size_t)128 * n_heads;        // float4s per slot
+  float m = -CUDART_INF_F, z = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = s0; s < s1; s += 4) {
+    float l[4];
+    float4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool in = s + k < s1;
+      l[k] = in ? __ldg(lse_part + (size_t)(s + k) * n_heads + h) : -CUDART_INF_F;
+      v[k] = in ? __ldg(src + (size_t)(s + k) * slot_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float m_new = fmaxf(m, fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3])));
+    if (m_new == -CUDART_INF_F) continue;
+    const float r = (m == -CUDART_INF_F) ? 0.f : __expf(m - m_new);
+    acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
+    z *= r;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float wgt = (l[k] == -CUDART_INF_F) ? 0.f : __expf(l[k] - m_new);
+      acc.x += wgt * v[k].x; acc.y += wgt * v[k].y; acc.z += wgt * v[k].z; acc.w += wgt * v[k].w;
+      z += wgt;
+    }
+    m = m_new;
   }
   const float inv_z = z > 0.f ? 1.f / z : 0.f;
-
-  const int g = blockIdx.y * (kCombineCols / 4) + grp;   // this thread's 4-column group
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int s = s0; s < s1; ++s) {
-    const float l = __ldg(lse_part + (size_t)s * n_heads + h);
-    const float wgt = (l == -CUDART_INF_F) ? 0.f : __expf(l - lmax) * inv_z;
-    const float4 v = __ldg(reinterpret_cast<const float4*>(o_part) + ((size_t)s * 128 + g) * n_heads + h);
-    acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
-  }
   *reinterpret_cast<uint2*>(o_lat + ((size_t)n * n_heads + h) * 512 + 4 * g) =
-      make_uint2(ptx::pack_bf16(acc.x, acc.y), ptx::pack_bf16(acc.z, acc.w));
+      make_uint2(ptx::pack_bf16(acc.x * inv_z, acc.y * inv_z), ptx::pack_bf16(acc.z * inv_z, acc.w * inv_z));
   if (lse_out && blockIdx.y == 0 && grp == 0)
-    lse_out[(size_t)n * n_heads + h] = z > 0.f ? lmax + __logf(z) : -CUDART_INF_F;
+    lse_out[(size_t)n * n_heads + h] = z > 0.f ? m + __logf(z) : -CUDART_INF_F;
 }
 
 __global__ void mla_gather_pages_kernel(const uint4* __restrict__ pool, const int32_t* __restrict__ bt,
