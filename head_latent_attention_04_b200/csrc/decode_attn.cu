@@ -23,8 +23,10 @@
 // decisions.  Each CTA accumulates its 256 output columns.
 //
 // TMEM (512 columns): O [0,256) fp32, S [256,320) fp32 (released as soon as
-// the sender has read it), P [320,384) as two bf16 buffers (A operand of the
-// PV product), q_lat half [384,512) as bf16 pairs (A operand of QK).
+// the sender has read it), P [320,352) bf16 (A operand of the PV product),
+// q_lat half [352,480) and q_rope half [480,496) as bf16 pairs (A operands of
+// QK).  Shared memory holds five 36 KB stages of cache rows and one fp16 score
+// tile each way (own, peer); both tiles are read right after they land.
 //
 // Warp roles (480 threads): warp 0 TMA producer; warp 1 QK issuer and TMEM
 // owner; warp 2 PV issuer (two issuing threads, so a page waiting for its
@@ -50,19 +52,17 @@ using namespace ptx;
 
 constexpr int kPage = 64;
 constexpr int kRows = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kChunkBytes = kPage * 128;                     // 64 keys x 64 latent cols (SW128)
 constexpr int kRopeBytes = kPage * 64;                       // 64 keys x 32 rope cols (SW64)
 constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;    // 36 KB: half a page
-constexpr int kQRopeBytes = kRows * 64;                      // 128 rows x 32 rope cols (SW64)
 constexpr int kXRow = 64 * 2;                                // fp16 score row, 16B chunks XOR (row & 7)
 constexpr int kXBytes = kRows * kXRow;                       // one score tile (16 KB)
 
 constexpr int kOffKV = 0;
-constexpr int kOffQRope = kOffKV + kStages * kStageBytes;
-constexpr int kOffXPeer = kOffQRope + kQRopeBytes;      // peer's partial scores, 2 tiles
-constexpr int kOffXOwn = kOffXPeer + 2 * kXBytes;       // own partial scores (fp16), 2 tiles
-constexpr int kOffPMax = kOffXOwn + 2 * kXBytes;        // fp32 [2 pages][2 halves][128] half-row maxima
+constexpr int kOffXPeer = kOffKV + kStages * kStageBytes;   // peer's partial scores (one tile)
+constexpr int kOffXOwn = kOffXPeer + kXBytes;                // own partial scores (fp16, one tile)
+constexpr int kOffPMax = kOffXOwn + kXBytes;                 // fp32 [2 pages][2 halves][128] half-row maxima
 constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;      // fp32 [2 items][2 halves][128] half-row sums
 constexpr int kOffBar = kOffLSum + 4 * kRows * 4;
 
@@ -70,12 +70,13 @@ constexpr int kThreads = 480;            // 15 warps
 constexpr int kSenderWarp0 = 3, kSoftWarp0 = 7;
 constexpr int kSoftWarps = 8;
 
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 384, kTmemCols = 512;
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemQR = 480, kTmemCols = 512;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 
 struct DecodeParams {
   const __nv_bfloat16* q_lat;   // [N][H][512]
+  const __nv_bfloat16* q_rope;  // [N][H][64]
   const int32_t* block_table;   // [B][max_blocks]
   const int32_t* seq_lens;      // [B]
   const int32_t* plan;
@@ -93,12 +94,11 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t s_full;       // QK product of the current page is in S
   uint64_t s_read;       // the sender has read S (the next QK may overwrite it)
-  uint64_t own_full[2];  // own fp16 partial-score tile b written (4 sender warps)
-  uint64_t own_free[2];  // own tile b consumed by the softmax (8 warps) and read by its bulk copy (1)
-  uint64_t x_recv[2];    // peer's fp16 partial scores landed in tile b (1 arrival + 16 KB tx)
-  uint64_t x_sendok[2];  // peer has consumed its tile b, which this CTA may refill (8 remote arrivals)
-  uint64_t p_full[2];    // P buffer b written (O rescaled if needed), 8 softmax warps
-  uint64_t p_free[2];    // PV product that read P buffer b is complete
+  uint64_t own_full;     // own fp16 partial-score tile written (4 sender warps)
+  uint64_t own_free;     // own tile read by the softmax (8 warps) and by its bulk copy (1)
+  uint64_t x_recv;       // peer's fp16 partial scores landed in the peer tile (1 arrival + 16 KB tx)
+  uint64_t x_sendok;     // peer has read its peer tile, which this CTA may refill (8 remote arrivals)
+  uint64_t p_full;       // P written (O rescaled if needed), 8 softmax warps
   uint64_t o_full;        // PV product of a page complete (awaited one page behind, for rescaling)
   uint64_t o_done;        // every PV product of the current item complete (epilogue)
   uint64_t o_free, qk_done, pv_done;
@@ -128,11 +128,10 @@ __device__ __forceinline__ float ex2(float x) {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rope,
-                  const __grid_constant__ CUtensorMap tm_qrope, const DecodeParams p) {
+                  const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_kv = smem + kOffKV;
-  uint8_t* s_qrope = smem + kOffQRope;
   uint8_t* s_xpeer = smem + kOffXPeer;
   uint8_t* s_xown = smem + kOffXOwn;
   float* s_pmax = reinterpret_cast<float*>(smem + kOffPMax);
@@ -151,19 +150,16 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    mbar_init(&bars->q_full, 1 + 4);   // q_rope TMA + the 4 q_lat loader warps
+    mbar_init(&bars->q_full, 4);       // the 4 q_lat / q_rope loader warps
     mbar_init(&bars->q_empty, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_read, 4);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->own_full[b], 4);
-      mbar_init(&bars->own_free[b], kSoftWarps + 1);
-      mbar_init(&bars->x_recv[b], 1);
-      mbar_init(&bars->x_sendok[b], kSoftWarps);
-      mbar_init(&bars->p_full[b], kSoftWarps);
-      mbar_init(&bars->p_free[b], 1);
-    }
-    for (int b = 0; b < 2; ++b) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);   // armed for pages 0, 1
+    mbar_init(&bars->own_full, 4);
+    mbar_init(&bars->own_free, kSoftWarps + 1);
+    mbar_init(&bars->x_recv, 1);
+    mbar_init(&bars->x_sendok, kSoftWarps);
+    mbar_init(&bars->p_full, kSoftWarps);
+    mbar_arrive_expect_tx(&bars->x_recv, kXBytes);   // armed for page 0
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, kSoftWarps);
@@ -178,7 +174,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     fence_mbar_init();
     prefetch_tmap(&tm_kv);
     prefetch_tmap(&tm_rope);
-    prefetch_tmap(&tm_qrope);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -214,20 +209,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     bool fail = false;
     for (int it = it_begin; it < it_end && !fail && !*abort_flag; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
-      const int b = w[kItB], row = w[kItRow], pb = w[kItPageBegin], pe = w[kItPageEnd];
-      const int ii = it - it_begin;
-      if (lane == 0) {
-        if (ii > 0 && !mbar_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) {
-          fail = true;
-        } else {
-          mbar_arrive_expect_tx(&bars->q_full, kQRopeBytes);
-          tma_load_3d(s_qrope, &tm_qrope, &bars->q_full, 32 * rank, 0, row);
-          if (it + 1 < it_end)   // the next item's q_lat rows, so that its loader reads them from L2
-            bulk_prefetch_l2(p.q_lat + (size_t)items[(size_t)(it + 1) * kItemWords + kItRow] * p.n_heads * 512,
-                             (uint32_t)p.n_heads * 1024u);
-        }
+      const int b = w[kItB], pb = w[kItPageBegin], pe = w[kItPageEnd];
+      if (lane == 0 && it + 1 < it_end) {   // the next item's query rows, so that its loaders read them from L2
+        const size_t nrow = (size_t)items[(size_t)(it + 1) * kItemWords + kItRow];
+        bulk_prefetch_l2(p.q_lat + nrow * p.n_heads * 512, (uint32_t)p.n_heads * 1024u);
+        bulk_prefetch_l2(p.q_rope + nrow * p.n_heads * 64, (uint32_t)p.n_heads * 128u);
       }
-      fail = __shfl_sync(0xffffffffu, fail, 0);
       int my_blk = 0;
       for (int pg = pb; pg < pe && !fail; ++pg, ++g) {
         const int rel = pg - pb;
@@ -276,7 +263,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
       const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
       const uint64_t kr_desc0 = sdesc(smem_u32(s_kv) + 4 * kChunkBytes, 16, 512, kSwizzle64B);
-      const uint64_t qr_desc = sdesc(smem_u32(s_qrope), 16, 512, kSwizzle64B);
       bool ok = true;
       int g = 0;
       for (int it = it_begin; ok && it < it_end; ++it) {
@@ -298,11 +284,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * t,
                    kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
 #pragma unroll
-          for (int t = 0; t < 2; ++t)    // RoPE half: K = 32
-            mma_ss(tmem + kTmemS, qr_desc + (uint64_t)(t * 2), krd + (uint64_t)(t * 2), idesc_qk, 1);
+          for (int t = 0; t < 2; ++t)    // RoPE half: K = 32, A = q_rope from TMEM
+            mma_ts(tmem + kTmemS, tmem + kTmemQR + 8 * t, krd + (uint64_t)(t * 2), idesc_qk, 1);
           mma_commit(&bars->s_full);
         }
-        if (ok) mma_commit(&bars->q_empty);   // q_lat (TMEM) and q_rope (smem) may be replaced
+        if (ok) mma_commit(&bars->q_empty);   // q_lat and q_rope (TMEM) may be replaced
       }
       if (!ok) {
         *abort_flag = 1;
@@ -325,8 +311,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         const int n = w[kItPageEnd] - w[kItPageBegin];
         const int ii = it - it_begin;
         for (int j = 0; j < n; ++j, ++g) {
-          const int s = g % kStages, b = g & 1;
-          if (!mbar_wait(&bars->p_full[b], (g >> 1) & 1, abort_flag) ||
+          const int s = g % kStages;
+          if (!mbar_wait(&bars->p_full, g & 1, abort_flag) ||
               (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, abort_flag))) {
             ok = false;
             break;
@@ -335,9 +321,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           const uint64_t vd = v_desc0 + (uint64_t)((s * kStageBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16; P (bf16 pairs) from TMEM
-            mma_ts(tmem + kTmemO, tmem + kTmemP + 32 * b + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+            mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
                    (j | kk) != 0);
-          mma_commit(&bars->p_free[b]);
           mma_commit(&bars->kv_empty[s]);
           mma_commit(&bars->o_full);
         }
@@ -353,22 +338,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mbar_wait(&bars->pv_done, 0, nullptr);
     }
   } else if (warp < kSoftWarp0) {
-    // ------------------------------------------------------------ q_lat loader and score sender (4 warps)
-    // At each item start the thread of row r copies its 256 q_lat columns
-    // into TMEM (A operand of the QK product) once the previous item's last
-    // QK has completed; the producer has prefetched those rows into L2.
-    // Reads this CTA's partial scores (its 288 columns) as soon as the QK
-    // product lands, frees S, rounds to fp16 into the local own-tile b, and
-    // one thread pushes that tile to the peer's tile b with a bulk copy that
-    // completes on the peer's x_recv[b].  Thread = one row, 64 keys; 16-byte
-    // chunks XOR-swizzled by (row & 7).  (Per-thread st.async stores into
-    // the peer raced with the peer's reads under load; the bulk copy is
-    // deterministic.)
+    // ------------------------------------------------------------ query loader and score sender (4 warps)
+    // At each item start the thread of row r copies its 256 q_lat columns and
+    // its 32 q_rope columns into TMEM (A operands of the QK product) once the
+    // previous item's last QK has completed; the producer has prefetched those
+    // rows into L2.  Per page it reads this CTA's partial scores (its 288
+    // columns) as soon as the QK product lands, frees S, rounds to fp16 into
+    // the own tile, and one thread pushes that tile to the peer's tile with a
+    // bulk copy that completes on the peer's x_recv.  Thread = one row, 64
+    // keys; 16-byte chunks XOR-swizzled by (row & 7).  (Per-thread st.async
+    // stores into the peer raced with the peer's reads under load; the bulk
+    // copy is deterministic.)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t x_peer = mapa(smem_u32(s_xpeer), peer);
-    const uint32_t x_recv_peer = mapa(smem_u32(&bars->x_recv[0]), peer);
+    const uint32_t x_recv_peer = mapa(smem_u32(&bars->x_recv), peer);
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
@@ -389,13 +374,23 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
         }
+        {
+          const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + ((size_t)w[kItRow] * p.n_heads + r) * 64 +
+                                                             32 * rank);
+          uint32_t v[16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 q = r < p.n_heads ? __ldg(rsrc + k) : make_uint4(0, 0, 0, 0);
+            v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
+          }
+          tmem_st16(tmem + lane_addr + kTmemQR, v);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_full);
       }
       for (int j = 0; j < n; ++j, ++g) {
-        const int b = g & 1;
         uint32_t v[64];
         if (!warp_wait(&bars->s_full, g & 1, abort_flag)) goto sender_fail;
         tc_fence_after();
@@ -408,10 +403,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         uint32_t hv[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) hv[k] = pack_f16(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
-        if (g >= 2 && !warp_wait(&bars->own_free[b], ((g >> 1) - 1) & 1, abort_flag)) goto sender_fail;
-        if (g >= 2 && !warp_wait(&bars->x_sendok[b], ((g >> 1) - 1) & 1, abort_flag)) goto sender_fail;
+        // single tile: page g - 1's own tile must have been read by the softmax and the copy
+        if (g >= 1 && !warp_wait(&bars->own_free, (g - 1) & 1, abort_flag)) goto sender_fail;
         {
-          uint8_t* own = s_xown + b * kXBytes + r * kXRow;
+          uint8_t* own = s_xown + r * kXRow;
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             *reinterpret_cast<uint4*>(own + ((k ^ (r & 7)) << 4)) =
@@ -419,15 +414,18 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         }
         fence_proxy_async_smem();   // the bulk copy below reads the tile through the async proxy
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->own_full[b]);
+        if (lane == 0) mbar_arrive(&bars->own_full);
         if (warp == kSenderWarp0 && lane == 0) {
-          // one bulk copy of the whole tile to the peer, completing on its x_recv[b];
+          // one bulk copy of the whole tile to the peer, completing on its x_recv;
           // the local tile may be rewritten only after the copy has read it
-          if (!mbar_wait(&bars->own_full[b], (g >> 1) & 1, abort_flag)) goto sender_fail;
-          bulk_copy_to_peer(x_peer + b * kXBytes, smem_u32(s_xown + b * kXBytes), kXBytes, x_recv_peer + 8 * b);
+          // and the peer must have read page g - 1 out of its peer tile
+          if (!mbar_wait(&bars->own_full, g & 1, abort_flag) ||
+              (g >= 1 && !mbar_wait(&bars->x_sendok, (g - 1) & 1, abort_flag)))
+            goto sender_fail;
+          bulk_copy_to_peer(x_peer, smem_u32(s_xown), kXBytes, x_recv_peer);
           bulk_commit();
           bulk_wait_read<0>();
-          mbar_arrive(&bars->own_free[b]);
+          mbar_arrive(&bars->own_free);
         }
       }
     }
@@ -445,7 +443,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
-    const uint32_t x_sendok_peer = mapa(smem_u32(&bars->x_sendok[0]), peer);
+    const uint32_t x_sendok_peer = mapa(smem_u32(&bars->x_sendok), peer);
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
@@ -456,22 +454,42 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       float m_ref = -CUDART_INF_F, l_run = 0.f;
       for (int j = 0; j < n; ++j) {
         const int gj = g + j, b = gj & 1;
-        // full score = fp16(own partial) + fp16(peer partial), identical in both CTAs
-        if (!warp_wait(&bars->own_full[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
-        if (!warp_wait_cluster(&bars->x_recv[b], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
+        // full score = fp16(own partial) + fp16(peer partial), identical in both CTAs.
+        // The own tile is read (and released) first: it lands before the peer's.
         uint4 po[4], pr[4];
+        uint32_t used = 0;
+        const uint32_t off_base = (uint32_t)(4 * c);
+        if (!warp_wait(&bars->own_full, gj & 1, abort_flag)) goto softmax_fail;
         {
-          const uint8_t* orow = s_xown + b * kXBytes + r * kXRow;
-          const uint8_t* xrow = s_xpeer + b * kXBytes + r * kXRow;
+          const uint8_t* orow = s_xown + r * kXRow;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint32_t off = (uint32_t)(((4 * c + k) ^ (r & 7)) << 4);
-            po[k] = *reinterpret_cast<const uint4*>(orow + off);
-            pr[k] = *reinterpret_cast<const uint4*>(xrow + off);
+            po[k] = *reinterpret_cast<const uint4*>(orow + (((off_base + k) ^ (r & 7)) << 4));
+            used |= po[k].x ^ po[k].w;
+          }
+          uint32_t bar_addr = smem_u32(&bars->own_free);
+          asm volatile("" : "+r"(bar_addr) : "r"(used));   // arrive only after the own tile was read
+          __syncwarp();
+          if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_addr) : "memory");
+        }
+        if (!warp_wait_cluster(&bars->x_recv, gj & 1, abort_flag)) goto softmax_fail;
+        {
+          const uint8_t* xrow = s_xpeer + r * kXRow;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            pr[k] = *reinterpret_cast<const uint4*>(xrow + (((off_base + k) ^ (r & 7)) << 4));
+            used |= pr[k].x ^ pr[k].w;
+          }
+          // the peer tile is consumed: re-arm x_recv for page gj + 1, then let the peer refill it
+          uint32_t ok_addr = x_sendok_peer;
+          asm volatile("" : "+r"(ok_addr) : "r"(used));   // issue only after the tile was read
+          __syncwarp();
+          if (lane == 0) {
+            if (warp == kSoftWarp0) mbar_arrive_expect_tx(&bars->x_recv, kXBytes);
+            mbar_arrive_relaxed_cluster(ok_addr);
           }
         }
         float sc[32];
-        uint32_t used = 0;
         {
           const uint32_t* ow = reinterpret_cast<const uint32_t*>(po);
           const uint32_t* pw = reinterpret_cast<const uint32_t*>(pr);
@@ -479,20 +497,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           for (int k = 0; k < 16; ++k) {
             const float2 a = unpack_f16x2(ow[k]);
             const float2 o = unpack_f16x2(pw[k]);
-            used |= pw[k] ^ ow[k];
             sc[2 * k] = a.x + o.x;
             sc[2 * k + 1] = a.y + o.y;
-          }
-        }
-        // both tiles b are consumed: re-arm x_recv[b] for page gj + 2, then release the tiles
-        {
-          uint32_t ok_addr = x_sendok_peer + 8 * b;
-          asm volatile("" : "+r"(ok_addr) : "r"(used));   // issue only after the tiles were read
-          __syncwarp();
-          if (lane == 0) {
-            if (warp == kSoftWarp0) mbar_arrive_expect_tx(&bars->x_recv[b], kXBytes);
-            mbar_arrive(&bars->own_free[b]);
-            mbar_arrive_relaxed_cluster(ok_addr);
           }
         }
         const int tok0 = (pb + j) * kPage + 32 * c;
@@ -539,8 +545,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         }
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
-        // P buffer b is free once the PV product two pages back has completed
-        if (gj >= 2 && !warp_wait(&bars->p_free[b], ((gj >> 1) - 1) & 1, abort_flag)) goto softmax_fail;
+        // the single P buffer is free once the previous page's PV product has completed
+        if (gj >= 1 && !warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
         if (__any_sync(0xffffffffu, move && j > 0)) {
           if (!warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
           tc_fence_after();
@@ -556,11 +562,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           }
           tmem_st_wait();
         }
-        tmem_st16(tmem + lane_addr + kTmemP + 32 * b + 16 * c, pk);   // keys [32c, 32c+32) as bf16 pairs
+        tmem_st16(tmem + lane_addr + kTmemP + 16 * c, pk);   // keys [32c, 32c+32) as bf16 pairs
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[b]);
+        if (lane == 0) mbar_arrive(&bars->p_full);
       }
 
       // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot
@@ -646,7 +652,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
                                 const int32_t* seq_lens, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream) {
-  CUtensorMap tm_kv, tm_rope, tm_q;
+  CUtensorMap tm_kv, tm_rope;
   const uint64_t pdims[2] = {576, (uint64_t)d.num_blocks * kPage};
   const uint64_t pstr[1] = {576 * 2};
   const uint32_t box_kv[2] = {64, kPage};
@@ -656,14 +662,10 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
   st = encode_tmap_bf16(&tm_rope, kv_pool, 2, pdims, pstr, box_rope, CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != MLA_OK) return st;
   const int N = d.B * d.s_q;
-  const uint64_t qdims[3] = {64, (uint64_t)d.n_heads, (uint64_t)N};
-  const uint64_t qstr[2] = {64 * 2, (uint64_t)d.n_heads * 64 * 2};
-  const uint32_t box_q[3] = {32, kRows, 1};
-  st = encode_tmap_bf16(&tm_q, q_rope, 3, qdims, qstr, box_q, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (st != MLA_OK) return st;
 
   DecodeParams p;
   p.q_lat = static_cast<const __nv_bfloat16*>(q_lat);
+  p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.plan = plan_dev;
@@ -684,8 +686,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
 
   cudaError_t e = decode_smem_attr();
   if (e == cudaSuccess) {
-    e = launch_pdl(mla_decode_kernel, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv, tm_rope,
-                   tm_q, p);
+    e = launch_pdl(mla_decode_kernel, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv, tm_rope, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
