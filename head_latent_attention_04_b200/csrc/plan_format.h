@@ -9,10 +9,11 @@ namespace mla {
 constexpr int32_t kPlanMagic = 0x314C414D;  // "MLA1" little-endian
 constexpr int kPlanHeaderWords = 16;
 constexpr int kItemWords = 8;
-// Planner cost of starting a work item, in pages: loading the row's q_lat
-// into TMEM and writing its output take about as long as three pages of the
-// attention pipeline.
-constexpr int32_t kItemCostPages = 3;
+// Planner cost of starting a work item, in pages: loading the row's query
+// into TMEM, refilling the pipeline and writing the output take about as long
+// as five pages of the attention pipeline (measured per-cluster finish times:
+// 4.5 to 5.6 pages per extra item across the benchmark workloads).
+constexpr int32_t kItemCostPages = 5;
 
 enum PlanHeader : int {
   kHdrMagic = 0,

@@ -108,7 +108,7 @@ mla_status_t mla_out_uv(const void* o_lat, const void* w_uv, void* out,
  * persistent grid of 2-CTA clusters; each cluster walks a contiguous range of
  * the flattened (sequence, page) work list of one query position, so a long
  * sequence is split across clusters and a cluster can cover several short
- * ones.  Ranges are equal in pages plus a fixed cost of three pages for every
+ * ones.  Ranges are equal in pages plus a fixed cost of five pages for every
  * row a range starts.  Pieces of a split row are merged by mla_combine.
  *
  * mla_plan_size: upper bounds for the plan (int32 words, in bytes) and for

@@ -23,7 +23,7 @@ def test_library_exports_every_declared_symbol():
 
 
 # ------------------------------------------------------------------ independent planner
-ITEM_COST_PAGES = 3
+ITEM_COST_PAGES = 5
 
 
 def py_plan(seq_lens, s_q, causal, n_heads, num_clusters, page=64):
