@@ -10,10 +10,14 @@
 // writes: element (slot, h, col) of O_i sits at
 //   ((slot * 128 + col / 4) * n_heads + h) * 4 + col % 4,
 // so that 32 consecutive heads of one 4-column group are 512 contiguous bytes.
-// HBM-bound: a block takes one row and 16 columns; thread (h, group) reads one
-// 4-column group of every piece (consecutive h -> coalesced 16-byte loads) and
-// writes 4 bf16 of its head.  Small grids (few rows cut into many pieces) still
-// get N x 32 blocks; the pieces are merged in one pass, four at a time.
+// HBM-bound.  Thread (h, grp) of a block merges column groups
+// grp, grp + 4, ... (G of them) of one row, with consecutive h reading
+// consecutive 16-byte words (coalesced).  The pieces are merged in one pass,
+// P at a time with all their loads in flight.  G is picked on the host so that
+// the grid is about one wave of the SMs (few rows: small G, many blocks; many
+// rows: large G, up to 4), and P = 8 / G, so that every thread keeps 8 words
+// in flight and two blocks fit on an SM.  Blocks of rows that were not split
+// exit at once.
 #include "mla_internal.h"
 #include "plan_format.h"
 #include "ptx.cuh"
@@ -24,10 +28,10 @@
 namespace mla {
 namespace {
 
-constexpr int kCombineThreads = 512;   // 128 heads x 4 column groups
-constexpr int kCombineCols = 16;       // columns per block
+constexpr int kCombineThreads = 512;   // 128 heads x 4 column-group lanes
 
-__global__ void __launch_bounds__(kCombineThreads)
+template <int G, int P>
+__global__ void __launch_bounds__(kCombineThreads, 2)
 mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o_part,
                    const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o_lat,
                    float* __restrict__ lse_out, int n_heads) {
@@ -41,38 +45,56 @@ mla_combine_kernel(const int32_t* __restrict__ plan, const float* __restrict__ o
   const int s0 = rs[n], s1 = rs[n + 1];
   if (s1 <= s0) return;   // row written whole by the attention kernel
 
-  // One pass over the pieces, four at a time with all their loads in flight,
-  // keeping a running maximum of the LSEs and rescaling the sums when it grows.
-  const int g = blockIdx.y * (kCombineCols / 4) + grp;   // this thread's 4-column group
-  const float4* src = reinterpret_cast<const float4*>(o_part) + (size_t)g * n_heads + h;
+  // Column group of lane i: g0 + 4 i.  Running maximum of the LSEs, sums
+  // rescaled when it grows.
+  const int g0 = blockIdx.y * (4 * G) + grp;
+  const float4* src = reinterpret_cast<const float4*>(o_part) + (size_t)g0 * n_heads + h;
   const size_t slot_stride = (size_t)128 * n_heads;        // float4s per slot
+  const size_t lane_stride = (size_t)4 * n_heads;          // float4s between this thread's groups
   float m = -CUDART_INF_F, z = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = s0; s < s1; s += 4) {
-    float l[4];
-    float4 v[4];
+  float4 acc[G];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+  for (int i = 0; i < G; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = s0; s < s1; s += P) {
+    float l[P];
+    float4 v[P][G];
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
       const bool in = s + k < s1;
       l[k] = in ? __ldg(lse_part + (size_t)(s + k) * n_heads + h) : -CUDART_INF_F;
-      v[k] = in ? __ldg(src + (size_t)(s + k) * slot_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < G; ++i)
+        v[k][i] = in ? __ldg(src + (size_t)(s + k) * slot_stride + i * lane_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const float m_new = fmaxf(m, fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3])));
+    float lm = l[0];
+#pragma unroll
+    for (int k = 1; k < P; ++k) lm = fmaxf(lm, l[k]);
+    const float m_new = fmaxf(m, lm);
     if (m_new == -CUDART_INF_F) continue;
     const float r = (m == -CUDART_INF_F) ? 0.f : __expf(m - m_new);
-    acc.x *= r; acc.y *= r; acc.z *= r; acc.w *= r;
     z *= r;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int i = 0; i < G; ++i) {
+      acc[i].x *= r; acc[i].y *= r; acc[i].z *= r; acc[i].w *= r;
+    }
+#pragma unroll
+    for (int k = 0; k < P; ++k) {
       const float wgt = (l[k] == -CUDART_INF_F) ? 0.f : __expf(l[k] - m_new);
-      acc.x += wgt * v[k].x; acc.y += wgt * v[k].y; acc.z += wgt * v[k].z; acc.w += wgt * v[k].w;
       z += wgt;
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        acc[i].x += wgt * v[k][i].x; acc[i].y += wgt * v[k][i].y;
+        acc[i].z += wgt * v[k][i].z; acc[i].w += wgt * v[k][i].w;
+      }
     }
     m = m_new;
   }
   const float inv_z = z > 0.f ? 1.f / z : 0.f;
-  *reinterpret_cast<uint2*>(o_lat + ((size_t)n * n_heads + h) * 512 + 4 * g) =
-      make_uint2(ptx::pack_bf16(acc.x * inv_z, acc.y * inv_z), ptx::pack_bf16(acc.z * inv_z, acc.w * inv_z));
+  __nv_bfloat16* dst = o_lat + ((size_t)n * n_heads + h) * 512 + 4 * g0;
+#pragma unroll
+  for (int i = 0; i < G; ++i)
+    *reinterpret_cast<uint2*>(dst + 16 * i) =
+        make_uint2(ptx::pack_bf16(acc[i].x * inv_z, acc[i].y * inv_z), ptx::pack_bf16(acc[i].z * inv_z, acc[i].w * inv_z));
   if (lse_out && blockIdx.y == 0 && grp == 0)
     lse_out[(size_t)n * n_heads + h] = z > 0.f ? m + __logf(z) : -CUDART_INF_F;
 }
@@ -95,9 +117,19 @@ __global__ void mla_gather_pages_kernel(const uint4* __restrict__ pool, const in
 mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,
                             const float* o_part, const float* lse_part, void* o_lat,
                             float* lse_out, void* stream) {
-  dim3 grid(n_rows, 512 / kCombineCols);
-  cudaError_t e = launch_pdl(mla_combine_kernel, grid, dim3(kCombineThreads), 0, stream, plan_dev, o_part, lse_part,
-                             static_cast<__nv_bfloat16*>(o_lat), lse_out, d.n_heads);
+  // Column groups per thread: the smallest G with n_rows x 32 / G blocks within
+  // about one wave (2 blocks of 512 threads per SM on 148 SMs).
+  const long long wave = 2LL * 148;
+  int G = 1;
+  while (G < 4 && (long long)n_rows * (32 / G) > wave) G *= 2;
+  dim3 grid(n_rows, 32 / G);
+  auto bf = static_cast<__nv_bfloat16*>(o_lat);
+  cudaError_t e;
+  switch (G) {
+    case 1: e = launch_pdl(mla_combine_kernel<1, 8>, grid, dim3(kCombineThreads), 0, stream, plan_dev, o_part, lse_part, bf, lse_out, d.n_heads); break;
+    case 2: e = launch_pdl(mla_combine_kernel<2, 4>, grid, dim3(kCombineThreads), 0, stream, plan_dev, o_part, lse_part, bf, lse_out, d.n_heads); break;
+    default: e = launch_pdl(mla_combine_kernel<4, 2>, grid, dim3(kCombineThreads), 0, stream, plan_dev, o_part, lse_part, bf, lse_out, d.n_heads); break;
+  }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "combine launch: %s", cudaGetErrorString(e));
   return MLA_OK;
