@@ -22,7 +22,8 @@
 //   per SM.
 // out_uv_kernel: one CTA per (head, token tile); K = 512 streams through a ring
 //   of up to 8 stages, each 16 KB of W_UV (MN-major: v contiguous) plus the
-//   tokens' 64-wide o_lat chunk.
+//   tokens' 64-wide o_lat chunk.  The CTA prefetches its head's W_UV into L2
+//   before waiting for the merge kernel, so the weight read overlaps it.
 #include "mla_internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -177,6 +178,13 @@ out_uv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
   if (warp == 1) {
     tmem_alloc(tmem_slot, cols);
     tmem_relinquish();
+  }
+  // This head's W_UV slice (128 KB) into L2 while the previous kernel finishes:
+  // a prefetch moves no data into this CTA and reads nothing the previous
+  // kernel writes, so it may precede the dependency wait.
+  if (warp == 0 && lane < kChunks) {
+    tma_prefetch_l2_3d(&tm_w, 0, h, lane * kBK);
+    tma_prefetch_l2_3d(&tm_w, 64, h, lane * kBK);
   }
   tc_fence_before();
   __syncthreads();

@@ -231,6 +231,13 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
       : "memory");
 }
 // Hint: bring [gptr, gptr + bytes) into L2 (16-byte aligned, multiple of 16 bytes), in 16 KB pieces.
+// L2 prefetch of one tensor-map box (a hint: no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_prefetch_l2(const void* gptr, uint32_t bytes) {
   const char* c = static_cast<const char*>(gptr);
   for (uint32_t off = 0; off < bytes; off += 16384u) {

@@ -23,7 +23,8 @@ def mla():
 
 
 # ------------------------------------------------------------------ projections alone
-@pytest.mark.parametrize("N,H", [(1, 1), (2, 16), (37, 128), (256, 128), (300, 7)])
+# one token tile of 16 to 256 columns, and several tiles
+@pytest.mark.parametrize("N,H", [(1, 1), (2, 16), (37, 128), (64, 128), (100, 128), (128, 9), (256, 128), (300, 7)])
 def test_absorb_q_matches_oracle(mla, N, H):
     w = W.make_workload(1, 1, H, [1], seed=N + H)
     g = torch.Generator().manual_seed(N)
