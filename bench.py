@@ -58,23 +58,27 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--projections", default="bf16", choices=["bf16", "fp8"],
+                    help="absorb / out_uv as bf16 GEMMs or as FP8 (E4M3) block-quantised BMMs")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------------------- accounting
-def algorithmic(seq_lens, s_q, H, causal=True):
+def algorithmic(seq_lens, s_q, H, causal=True, weight_bytes=2):
     """Algorithmic bytes / FLOPs of the step and of the attention kernel.
 
     Per attended (query, key) pair: 2*h*(2*d_c + d_R) FLOPs (QK over 576 +
     PV over 512 per head).  Per cached token: 576 bf16 = 1152 B, read once
     and shared by all heads and all s_q query tokens of its sequence.
+    ``weight_bytes``: bytes per W_UK / W_UV element (1 for E4M3 codes, whose
+    scales add 4 bytes per 128 x 128 block).
     """
     T = np.asarray(seq_lens, dtype=np.int64)
     N = len(T) * s_q
     pairs = int(sum(int(t) - s_q + 1 + i if causal else int(t) for t in T for i in range(s_q)))
     cache = int(T.sum()) * 576 * 2
-    w_bytes = 2 * 512 * H * 128 * 2
+    w_bytes = 2 * 512 * H * 128 * weight_bytes + (2 * 4 * H * 4 if weight_bytes == 1 else 0)
     attn_flops = pairs * 2 * H * (2 * 512 + 64)
     bmm_flops = 2 * (2 * N * H * 128 * 512)
     q_in = N * H * (128 + 64) * 2
@@ -307,9 +311,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.set_device(dev)
     preset = W.PRESETS[args.config]
     w = W.preset_workload(args.config, device=dev, seed=dp.replica_seed(preset.seed, rank))
-    acc = algorithmic(w.seq_lens, w.s_q, w.n_heads)
+    fp8 = args.projections == "fp8"
+    acc = algorithmic(w.seq_lens, w.s_q, w.n_heads, weight_bytes=1 if fp8 else 2)
     bt = torch.as_tensor(w.block_table, device=dev)
     dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev)
+    if fp8:   # weights quantised once, outside the timed region (static, as the weights are)
+        dec.use_fp8_projections(w.w_uk, w.w_uv)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -445,10 +452,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     res = {
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (attention); e4m3 codes with fp32 block scales (projections)" if fp8 else "bf16",
+        "data": "synthetic",
         "config": dict(workload_config(args.config, w), parallelism=f"dp{world} (independent replicas)",
                        num_clusters=dec.num_clusters, split_slots=dec.num_slots,
-                       graph=used_graph),
+                       graph=used_graph, projections=args.projections),
         "cache_tbs": acc["cache_bytes"] * world / (ms * 1e-3) / 1e12,
         "attn_cache_tbs": acc["cache_bytes"] / (attn * 1e-3) / 1e12,
         "tflops": acc["step_flops"] * world / (ms * 1e-3) / 1e12,

@@ -41,9 +41,9 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-mla_status_t encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                              const uint64_t* strides_bytes, const uint32_t* box,
-                              CUtensorMapSwizzle swizzle) {
+static mla_status_t encode_tmap(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank,
+                                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                                CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(MLA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t d[5], s[4];
@@ -54,11 +54,22 @@ mla_status_t encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, cons
     e[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, s,
+  CUresult r = fn(map, type, (cuuint32_t)rank, const_cast<void*>(base), d, s,
                   b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MLA_OK;
+}
+
+mla_status_t encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                              const uint64_t* strides_bytes, const uint32_t* box,
+                              CUtensorMapSwizzle swizzle) {
+  return encode_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box, swizzle);
+}
+
+mla_status_t encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  return encode_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, rank, dims, strides_bytes, box, swizzle);
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -124,6 +135,60 @@ mla_status_t mla_out_uv(const void* o_lat, const void* w_uv, void* out, int32_t 
   MLA_TRY(check_ptr(w_uv, "w_uv"));
   MLA_TRY(check_ptr(out, "out"));
   return launch_out_uv(o_lat, w_uv, out, n_tokens, n_heads, stream);
+}
+
+mla_status_t mla_quantize_w_uk_fp8(const void* w_uk, int32_t n_heads, void* w_codes, float* w_scales,
+                                   void* stream) {
+  clear_error();
+  if (n_heads < 1 || n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
+  MLA_TRY(check_ptr(w_uk, "w_uk"));
+  MLA_TRY(check_ptr(w_codes, "w_codes"));
+  if (!w_scales) return set_error(MLA_ERR_INVALID_ARG, "w_scales is NULL");
+  return launch_quantize_weight_fp8(w_uk, n_heads, false, w_codes, w_scales, stream);
+}
+
+mla_status_t mla_quantize_w_uv_fp8(const void* w_uv, int32_t n_heads, void* w_codes, float* w_scales,
+                                   void* stream) {
+  clear_error();
+  if (n_heads < 1 || n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
+  MLA_TRY(check_ptr(w_uv, "w_uv"));
+  MLA_TRY(check_ptr(w_codes, "w_codes"));
+  if (!w_scales) return set_error(MLA_ERR_INVALID_ARG, "w_scales is NULL");
+  return launch_quantize_weight_fp8(w_uv, n_heads, true, w_codes, w_scales, stream);
+}
+
+mla_status_t mla_quantize_rows_fp8(const void* x, int64_t rows, int32_t cols, void* codes, float* scales,
+                                   void* stream) {
+  clear_error();
+  if (rows < 0) return set_error(MLA_ERR_INVALID_ARG, "rows must be >= 0");
+  if (cols < 128 || cols % 128 != 0) return set_error(MLA_ERR_UNSUPPORTED, "cols must be a positive multiple of 128");
+  if (rows == 0) return MLA_OK;
+  MLA_TRY(check_ptr(x, "x"));
+  MLA_TRY(check_ptr(codes, "codes"));
+  if (!scales) return set_error(MLA_ERR_INVALID_ARG, "scales is NULL");
+  return launch_quantize_rows_fp8(x, rows, cols, codes, scales, stream);
+}
+
+mla_status_t mla_absorb_q_fp8(const void* q_nope, const void* w_uk_codes, const float* w_uk_scales, void* q_lat,
+                              int32_t n_tokens, int32_t n_heads, void* stream) {
+  clear_error();
+  MLA_TRY(check_tokens(n_tokens, n_heads));
+  MLA_TRY(check_ptr(q_nope, "q_nope"));
+  MLA_TRY(check_ptr(w_uk_codes, "w_uk_codes"));
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  if (!w_uk_scales) return set_error(MLA_ERR_INVALID_ARG, "w_uk_scales is NULL");
+  return launch_absorb_q_fp8(q_nope, w_uk_codes, w_uk_scales, q_lat, n_tokens, n_heads, stream);
+}
+
+mla_status_t mla_out_uv_fp8(const void* o_lat, const void* w_uv_codes, const float* w_uv_scales, void* out,
+                            int32_t n_tokens, int32_t n_heads, void* stream) {
+  clear_error();
+  MLA_TRY(check_tokens(n_tokens, n_heads));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  MLA_TRY(check_ptr(w_uv_codes, "w_uv_codes"));
+  MLA_TRY(check_ptr(out, "out"));
+  if (!w_uv_scales) return set_error(MLA_ERR_INVALID_ARG, "w_uv_scales is NULL");
+  return launch_out_uv_fp8(o_lat, w_uv_codes, w_uv_scales, out, n_tokens, n_heads, stream);
 }
 
 mla_status_t mla_max_clusters(int32_t* num_clusters) {

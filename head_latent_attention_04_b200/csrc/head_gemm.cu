@@ -30,6 +30,8 @@
 
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 namespace mla {
 namespace {
 
@@ -270,6 +272,405 @@ mla_status_t weight_map(CUtensorMap* m, const void* base, int H, int box_k) {
   return encode_tmap_bf16(m, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// ----------------------------------------------------------------- FP8 (E4M3) block-quantised BMMs
+// "Lower latency and higher throughput with multi-node DeepSeek deployment",
+// sections "Quantization" and "MLA layer": weights carry one scale per
+// 128 x 128 block (quantised once, here by quantize_weight_kernel) and
+// activations one scale per 128-element vector along K, computed on the fly.
+// A block's scale is s = amax / 448 and a value's code is E4M3(x * (448 /
+// amax)), rounded to nearest even; an all-zero block takes s = 1.  Products of
+// a K-block are summed exactly-rounded in fp32 by the tensor cores and scaled
+// by s_act * s_weight afterwards.
+
+constexpr float kE4M3Max = 448.f;
+
+// 128 bf16 (16 x 16 bytes) -> 128 E4M3 codes (32 words, element 4j + i in byte
+// i of word j) and the vector's scale.
+__device__ __forceinline__ float quant128(const uint4 (&x)[16], uint32_t (&q)[32]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+  }
+  const float r = amax > 0.f ? __fdiv_rn(kE4M3Max, amax) : 1.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t w[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t a = w[2 * i], b = w[2 * i + 1];
+      q[2 * k + i] = cvt_e4m3x2(__fmul_rn(__uint_as_float(a << 16), r), __fmul_rn(__uint_as_float(a & 0xFFFF0000u), r)) |
+                     (cvt_e4m3x2(__fmul_rn(__uint_as_float(b << 16), r), __fmul_rn(__uint_as_float(b & 0xFFFF0000u), r)) << 16);
+    }
+  }
+  return amax > 0.f ? __fdiv_rn(amax, kE4M3Max) : 1.f;
+}
+
+__device__ __forceinline__ void load128(const __nv_bfloat16* src, uint4 (&x)[16]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) x[k] = __ldg(reinterpret_cast<const uint4*>(src) + k);
+}
+
+// Codes of one 128-byte row into a K-major SW128 tile (16-byte chunk c of row
+// r at chunk c ^ (r & 7)); the tile base is 1024-byte aligned.
+__device__ __forceinline__ void put_row_sw128(uint8_t* tile, int r, const uint32_t (&q)[32]) {
+  uint8_t* row = tile + r * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
+}
+
+// One 128 x 128 weight block (kb, h) of W [512][H][128] bf16 -> codes and
+// scales[h][kb].  kTransposed = false: codes [H][512][128] (W_UK: rows k,
+// K = d contiguous); true: codes [H][128][512] (W_UV: rows v, K = k contiguous).
+template <bool kTransposed>
+__global__ void __launch_bounds__(128) quantize_weight_kernel(const __nv_bfloat16* __restrict__ w, int n_heads,
+                                                              uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  __shared__ __align__(16) __nv_bfloat16 tile[128][128];
+  __shared__ float wmax[4];
+  const int kb = blockIdx.x, h = blockIdx.y, t = threadIdx.x;
+  uint4 x[16];
+  load128(w + ((size_t)(kb * 128 + t) * n_heads + h) * 128, x);
+  float amax = 0.f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    *reinterpret_cast<uint4*>(&tile[t][8 * k]) = x[k];
+    const uint32_t ws[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(ws[i] << 16)), fabsf(__uint_as_float(ws[i] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((t & 31) == 0) wmax[t >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  const float r = amax > 0.f ? __fdiv_rn(kE4M3Max, amax) : 1.f;
+  if (t == 0) scales[h * 4 + kb] = amax > 0.f ? __fdiv_rn(amax, kE4M3Max) : 1.f;
+  // thread t writes output row t of the block: W_UK row k = kb*128 + t (over d),
+  // or W_UV row v = t (over k in the block, read down the tile's column t)
+  uint8_t* dst = kTransposed ? codes + ((size_t)h * 128 + t) * 512 + kb * 128
+                             : codes + ((size_t)h * 512 + kb * 128 + t) * 128;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t wds[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float f[4];
+      if constexpr (kTransposed) {   // down column t of the tile (consecutive threads, consecutive banks)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) f[i] = __bfloat162float(tile[16 * c + 4 * j + i][t]);
+      } else {                       // this thread's own row, still in registers
+        const uint4 v = x[2 * c + j / 2];
+        const uint32_t a = (j & 1) ? v.z : v.x, b = (j & 1) ? v.w : v.y;
+        f[0] = __uint_as_float(a << 16); f[1] = __uint_as_float(a & 0xFFFF0000u);
+        f[2] = __uint_as_float(b << 16); f[3] = __uint_as_float(b & 0xFFFF0000u);
+      }
+      wds[j] = cvt_e4m3x2(__fmul_rn(f[0], r), __fmul_rn(f[1], r)) | (cvt_e4m3x2(__fmul_rn(f[2], r), __fmul_rn(f[3], r)) << 16);
+    }
+    reinterpret_cast<uint4*>(dst)[c] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  }
+}
+
+// Rows of 128-element vectors: x [rows][cols] bf16 -> codes [rows][cols] and
+// scales [rows][cols / 128], one thread per vector (the on-the-fly activation
+// quantisation of the BMM kernels, exposed on its own).
+__global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, long long n_vec,
+                                     uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_vec; i += (long long)gridDim.x * blockDim.x) {
+    uint4 v[16];
+    load128(x + i * 128, v);
+    uint32_t q[32];
+    scales[i] = quant128(v, q);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      reinterpret_cast<uint4*>(codes + i * 128)[c] = make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
+  }
+}
+
+// absorb, FP8: one CTA per (128-row tile of the head's W_UK codes, head, token
+// tile).  A = codes [128 k][128 d] (one TMA box, SW128); the tokens' q_nope rows
+// arrive by TMA as bf16 (two SW128 chunks of 64 d, as in the bf16 kernel) and
+// are quantised from shared memory into a SW128 code tile, four threads per
+// row (32 values each, the row maximum combined by shuffles; a token tile is a
+// multiple of 16 rows, so every warp is wholly in or out of the loop); K = 128
+// in 4 MMAs; epilogue D * s_w[h][tile] * s_q[token], staged over the dead
+// operands.  Token tiles of at most 128.
+__global__ void __launch_bounds__(128)
+absorb_q_fp8_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                    const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ w_scales, GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int bn = p.bn;
+  uint8_t* sA = smem;                           // 16 KB of weight codes
+  uint8_t* sX = sA + kATileBytes;               // 2 chunks x bn x 128 B of bf16 q_nope
+  uint8_t* sB = sX + 2 * bn * 128;              // bn x 128 B of codes
+  uint8_t* sOut = smem;                         // bf16 [bn][128], over the operands once the MMAs are done
+  const int region = (kATileBytes + 3 * bn * 128) > bn * 256 ? (kATileBytes + 3 * bn * 128) : bn * 256;
+  float* s_act = reinterpret_cast<float*>(smem + region);     // [bn]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_act + kMaxBN);
+  uint64_t* done = full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int mt = blockIdx.x, h = blockIdx.y, n0 = blockIdx.z * bn;
+  const uint32_t cols = tmem_cols_for(bn);
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_out);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();   // global memory only from here
+  griddep_launch_dependents();
+
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(full, kATileBytes + 2 * bn * 128);
+    tma_load_2d(sA, &tm_w, full, 0, h * 512 + mt * kBM);
+    tma_load_3d(sX, &tm_x, full, 0, h, n0);
+    tma_load_3d(sX + bn * 128, &tm_x, full, 64, h, n0);
+  }
+  const bool landed = __all_sync(0xffffffffu, mbar_wait(full, 0, abort_flag));   // warp-uniform: the loop shuffles
+  if (landed) {
+    // item i: row r = i / 4, values [32 qq, 32 qq + 32) with qq = i % 4 (chunk qq / 2,
+    // 16-byte pieces 4 (qq % 2) .. + 3 of that chunk's swizzled row)
+    for (int i = threadIdx.x; i < bn * 4; i += 128) {
+      const int r = i >> 2, qq = i & 3;
+      const uint8_t* row = sX + (qq >> 1) * bn * 128 + r * 128;
+      float v[32];
+      float amax = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(row + ((((qq & 1) * 4 + k) ^ (r & 7)) << 4));
+        const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * k + 2 * j] = __uint_as_float(ws[j] << 16);
+          v[8 * k + 2 * j + 1] = __uint_as_float(ws[j] & 0xFFFF0000u);
+          amax = fmaxf(amax, fmaxf(fabsf(v[8 * k + 2 * j]), fabsf(v[8 * k + 2 * j + 1])));
+        }
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const float rcp = amax > 0.f ? __fdiv_rn(kE4M3Max, amax) : 1.f;
+      uint32_t q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        q[j] = cvt_e4m3x2(__fmul_rn(v[4 * j], rcp), __fmul_rn(v[4 * j + 1], rcp)) |
+               (cvt_e4m3x2(__fmul_rn(v[4 * j + 2], rcp), __fmul_rn(v[4 * j + 3], rcp)) << 16);
+      uint8_t* crow = sB + r * 128;   // code pieces 2 qq and 2 qq + 1 of row r
+      *reinterpret_cast<uint4*>(crow + (((2 * qq) ^ (r & 7)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+      *reinterpret_cast<uint4*>(crow + (((2 * qq + 1) ^ (r & 7)) << 4)) = make_uint4(q[4], q[5], q[6], q[7]);
+      if (qq == 0) s_act[r] = amax > 0.f ? __fdiv_rn(amax, kE4M3Max) : 1.f;
+    }
+  }
+  fence_proxy_async_smem();   // the MMAs read the code tile through the async proxy
+  const bool all_landed = __syncthreads_and(landed);
+  if (warp == 1 && lane == 0) {
+    if (all_landed) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_e4m3(kBM, bn);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)   // K = 128 codes = 128 bytes per row, 32 per MMA
+        mma_ss_f8(tmem, sdesc(smem_u32(sA) + kk * 32, 16, 1024, kSwizzle128B),
+                  sdesc(smem_u32(sB) + kk * 32, 16, 1024, kSwizzle128B), idesc, kk != 0);
+    } else {
+      *abort_flag = 1;
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+  const bool ok = __syncthreads_and(mbar_wait(done, 0, abort_flag) && !*abort_flag);
+  tc_fence_after();
+  if (ok) {
+    const float s_w = w_scales[h * 4 + mt];
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(sOut);
+    const int m = warp * 32 + lane;
+    for (int c = 0; c < bn; c += 32) {
+      uint32_t rr[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, rr);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c + j < bn) o[(c + j) * kBM + m] = __float2bfloat16_rn(__uint_as_float(rr[j]) * (s_w * s_act[c + j]));
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tma_store_3d(&tm_out, sOut, mt * kBM, h, n0);
+      bulk_commit();
+      bulk_wait_all<0>();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  if (warp == 1) tmem_dealloc(tmem, cols);
+}
+
+// out_uv, FP8: one CTA per (head, token tile of at most 128).  A = the head's
+// W_UV codes [128 v][512 k] as four 16 KB K-blocks, B = the tokens' o_lat rows
+// quantised per 128-vector into four SW128 tiles, one TMEM accumulator per
+// K-block (4 x bn columns), epilogue sum_kb D_kb * s_w[h][kb] * s_o[token][kb].
+__global__ void __launch_bounds__(128)
+out_uv_fp8_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_out,
+                  const __nv_bfloat16* __restrict__ o_lat, const float* __restrict__ w_scales, GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int bn = p.bn;
+  uint8_t* sA = smem;                           // 4 x 16 KB
+  uint8_t* sB = sA + 4 * kATileBytes;           // 4 x bn x 128 B
+  uint8_t* sOut = smem;                         // bn x 256 B, over the weight tiles once the MMAs are done
+  float* s_act = reinterpret_cast<float*>(sB + 4 * bn * 128);   // [4][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_act + 4 * 128);
+  uint64_t* done = full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.y, n0 = blockIdx.z * bn;
+  const uint32_t cols = tmem_cols_for(bn);
+  if (threadIdx.x == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_out);
+  }
+  // the head's 64 KB of codes into L2 while the previous kernel finishes (a hint)
+  if (warp == 0 && lane < 4) tma_prefetch_l2_2d(&tm_w, lane * 128, h * 128);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 4 * cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(full, 4 * kATileBytes);
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) tma_load_2d(sA + kb * kATileBytes, &tm_w, full, kb * 128, h * 128);
+  }
+  for (int i = threadIdx.x; i < 128 * 4; i += 128) {   // vector (token r, K-block kb)
+    const int r = i >> 2, kb = i & 3, n = n0 + r;
+    if (r >= bn) {   // past the tile: a zero scale for the epilogue's padding columns
+      s_act[kb * 128 + r] = 0.f;
+      continue;
+    }
+    uint32_t q[32];
+    float sc = 0.f;
+    if (n < p.n_tokens) {
+      uint4 x[16];
+      load128(o_lat + ((size_t)n * p.n_heads + h) * 512 + kb * 128, x);
+      sc = quant128(x, q);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) q[j] = 0;
+    }
+    put_row_sw128(sB + kb * bn * 128, r, q);
+    s_act[kb * 128 + r] = sc;
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (warp == 1 && lane == 0) {
+    if (mbar_wait(full, 0, abort_flag)) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_e4m3(kBM, bn);
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss_f8(tmem + kb * cols, sdesc(smem_u32(sA + kb * kATileBytes) + kk * 32, 16, 1024, kSwizzle128B),
+                    sdesc(smem_u32(sB + kb * bn * 128) + kk * 32, 16, 1024, kSwizzle128B), idesc, kk != 0);
+    } else {
+      *abort_flag = 1;
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+  const bool ok = __syncthreads_and(mbar_wait(done, 0, abort_flag) && !*abort_flag);
+  tc_fence_after();
+  if (ok) {
+    float s_w[4];
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) s_w[kb] = w_scales[h * 4 + kb];
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(sOut);
+    const int m = warp * 32 + lane;
+    for (int c = 0; c < bn; c += 32) {
+      float acc[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + kb * cols + c, rr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = fmaf(__uint_as_float(rr[j]), s_w[kb] * s_act[kb * 128 + c + j], acc[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c + j < bn) o[(c + j) * kBM + m] = __float2bfloat16_rn(acc[j]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tma_store_3d(&tm_out, sOut, 0, h, n0);
+      bulk_commit();
+      bulk_wait_all<0>();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  if (warp == 1) tmem_dealloc(tmem, 4 * cols);
+}
+
+cudaError_t set_smem_attrs_fp8() {
+  static cudaError_t e = [] {
+    cudaError_t a = cudaFuncSetAttribute(absorb_q_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    cudaError_t b = cudaFuncSetAttribute(out_uv_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    return a != cudaSuccess ? a : b;
+  }();
+  return e;
+}
+
+// Token tile of at most `max_bn`, a multiple of 16, tiles of near-equal size.
+int token_tile_max(int n_tokens, int max_bn, int* n_tiles) {
+  const int tiles = (n_tokens + max_bn - 1) / max_bn;
+  const int per = (n_tokens + tiles - 1) / tiles;
+  *n_tiles = tiles;
+  return ((per + 15) / 16) * 16;
+}
+
+// Shared memory padded so that the CTAs sharing an SM never ask for more than
+// its 512 TMEM columns: at most 512 / tmem_cols of them fit by shared memory.
+int pad_smem_for_tmem(int smem, int tmem_cols) {
+  const int ctas = 512 / tmem_cols;
+  const int floor_bytes = kSmemPerSM / (ctas + 1) - 1024 + 1;
+  return smem < floor_bytes ? floor_bytes : smem;
+}
+
 }  // namespace
 
 mla_status_t launch_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, int n_tokens,
@@ -318,6 +719,79 @@ mla_status_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int n
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "out_uv launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_quantize_weight_fp8(const void* w, int n_heads, bool transposed, void* codes, float* scales,
+                                        void* stream) {
+  auto wb = static_cast<const __nv_bfloat16*>(w);
+  auto cs = static_cast<uint8_t*>(codes);
+  auto st = static_cast<cudaStream_t>(stream);
+  if (transposed) quantize_weight_kernel<true><<<dim3(4, n_heads), 128, 0, st>>>(wb, n_heads, cs, scales);
+  else quantize_weight_kernel<false><<<dim3(4, n_heads), 128, 0, st>>>(wb, n_heads, cs, scales);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "quantize_weight launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_quantize_rows_fp8(const void* x, long long rows, int cols, void* codes, float* scales,
+                                      void* stream) {
+  const long long n_vec = rows * (cols / 128);
+  if (n_vec == 0) return MLA_OK;
+  const long long blocks = (n_vec + 127) / 128;
+  quantize_rows_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), n_vec, static_cast<uint8_t*>(codes), scales);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "quantize_rows launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_absorb_q_fp8(const void* q_nope, const void* w_codes, const float* w_scales, void* q_lat,
+                                 int n_tokens, int n_heads, void* stream) {
+  int tiles = 1;
+  const int bn = token_tile_max(n_tokens, 128, &tiles);   // bf16 rows + codes stay within 3 CTAs per SM
+  CUtensorMap tw, tx, to;
+  const uint64_t wdims[2] = {128, (uint64_t)n_heads * 512};
+  const uint64_t wstr[1] = {128};
+  const uint32_t wbox[2] = {128, (uint32_t)kBM};
+  mla_status_t st = encode_tmap_u8(&tw, w_codes, 2, wdims, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st == MLA_OK) st = act_map(&tx, q_nope, 128, n_heads, n_tokens, 64, bn, false);
+  if (st == MLA_OK) st = act_map(&to, q_lat, 512, n_heads, n_tokens, kBM, bn, true);
+  if (st != MLA_OK) return st;
+  const int region = std::max(kATileBytes + 3 * bn * 128, bn * 256);
+  const int smem = pad_smem_for_tmem(1024 + region + kMaxBN * 4 + 64, (int)tmem_cols_for(bn));
+  GemmParams p{n_tokens, n_heads, bn, 0};
+  cudaError_t e = set_smem_attrs_fp8();
+  if (e == cudaSuccess) {
+    e = launch_pdl(absorb_q_fp8_kernel, dim3(512 / kBM, n_heads, tiles), dim3(128), smem, stream, tw, tx, to,
+                   w_scales, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "absorb_q_fp8 launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_out_uv_fp8(const void* o_lat, const void* w_codes, const float* w_scales, void* out,
+                               int n_tokens, int n_heads, void* stream) {
+  int tiles = 1;
+  const int bn = token_tile_max(n_tokens, 128, &tiles);   // 4 accumulators of bn columns
+  CUtensorMap tw, to;
+  const uint64_t wdims[2] = {512, (uint64_t)n_heads * 128};
+  const uint64_t wstr[1] = {512};
+  const uint32_t wbox[2] = {128, (uint32_t)kBM};
+  mla_status_t st = encode_tmap_u8(&tw, w_codes, 2, wdims, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st == MLA_OK) st = act_map(&to, out, 128, n_heads, n_tokens, kBM, bn, true);
+  if (st != MLA_OK) return st;
+  const int smem = pad_smem_for_tmem(1024 + 4 * kATileBytes + 4 * bn * 128 + 4 * 128 * 4 + 64,
+                                     4 * (int)tmem_cols_for(bn));
+  GemmParams p{n_tokens, n_heads, bn, 0};
+  cudaError_t e = set_smem_attrs_fp8();
+  if (e == cudaSuccess) {
+    e = launch_pdl(out_uv_fp8_kernel, dim3(1, n_heads, tiles), dim3(128), smem, stream, tw, to,
+                   static_cast<const __nv_bfloat16*>(o_lat), w_scales, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "out_uv_fp8 launch: %s", cudaGetErrorString(e));
   return MLA_OK;
 }
 

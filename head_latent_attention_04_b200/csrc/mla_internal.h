@@ -41,6 +41,14 @@ mla_status_t launch_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, 
                              int n_heads, void* stream);
 mla_status_t launch_out_uv(const void* o_lat, const void* w_uv, void* out, int n_tokens,
                            int n_heads, void* stream);
+mla_status_t launch_quantize_weight_fp8(const void* w, int n_heads, bool transposed, void* codes, float* scales,
+                                        void* stream);
+mla_status_t launch_quantize_rows_fp8(const void* x, long long rows, int cols, void* codes, float* scales,
+                                      void* stream);
+mla_status_t launch_absorb_q_fp8(const void* q_nope, const void* w_codes, const float* w_scales, void* q_lat,
+                                 int n_tokens, int n_heads, void* stream);
+mla_status_t launch_out_uv_fp8(const void* o_lat, const void* w_codes, const float* w_scales, void* out,
+                               int n_tokens, int n_heads, void* stream);
 mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
                                 const void* kv_pool, const int32_t* block_table,
                                 const int32_t* seq_lens, const int32_t* plan_dev,

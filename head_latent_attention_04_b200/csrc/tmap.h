@@ -12,5 +12,8 @@ namespace mla {
 mla_status_t encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                               const uint64_t* strides_bytes, const uint32_t* box,
                               CUtensorMapSwizzle swizzle);
+// The same for bytes (8-bit codes).
+mla_status_t encode_tmap_u8(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                            const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle);
 
 }  // namespace mla

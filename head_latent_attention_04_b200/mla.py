@@ -26,7 +26,9 @@ MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_TIMEOUT = 3, 4, 5
 STATUS_BAD_BLOCK, STATUS_TIMEOUT, STATUS_BAD_SEQLEN = 0x1, 0x2, 0x4
 EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
-           "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes")
+           "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes",
+           "mla_quantize_w_uk_fp8", "mla_quantize_w_uv_fp8", "mla_quantize_rows_fp8", "mla_absorb_q_fp8",
+           "mla_out_uv_fp8")
 
 
 class MlaDims(ctypes.Structure):
@@ -51,6 +53,11 @@ for _name, _args in {
     "mla_combine": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_debug_gather_pages": [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "mla_decode_attn_combine_noalloc": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _vp, _vp, _vp, _vp],
+    "mla_quantize_w_uk_fp8": [_vp, _i32, _vp, _vp, _vp],
+    "mla_quantize_w_uv_fp8": [_vp, _i32, _vp, _vp, _vp],
+    "mla_quantize_rows_fp8": [_vp, ctypes.c_int64, _i32, _vp, _vp, _vp],
+    "mla_absorb_q_fp8": [_vp, _vp, _vp, _vp, _i32, _i32, _vp],
+    "mla_out_uv_fp8": [_vp, _vp, _vp, _vp, _i32, _i32, _vp],
 }.items():
     getattr(_lib, _name).argtypes = _args
     getattr(_lib, _name).restype = _i32
@@ -137,6 +144,62 @@ def out_uv(o_lat: torch.Tensor, w_uv: torch.Tensor, out: torch.Tensor | None = N
     return out
 
 
+@dataclass
+class Fp8Weight:
+    """A projection weight as E4M3 codes (uint8) and fp32 block scales [H][4]."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+
+
+def quantize_w_uk_fp8(w_uk: torch.Tensor, stream=None) -> Fp8Weight:
+    """W_UK bf16 [512][H][128] -> codes [H][512][128] and scales [H][4]."""
+    H = w_uk.shape[1]
+    codes = torch.empty((H, 512, 128), dtype=torch.uint8, device=w_uk.device)
+    scales = torch.empty((H, 4), dtype=torch.float32, device=w_uk.device)
+    _check(_lib.mla_quantize_w_uk_fp8(_ptr(w_uk), H, _ptr(codes), _ptr(scales), _stream(stream)),
+           "mla_quantize_w_uk_fp8")
+    return Fp8Weight(codes, scales)
+
+
+def quantize_w_uv_fp8(w_uv: torch.Tensor, stream=None) -> Fp8Weight:
+    """W_UV bf16 [512][H][128] -> codes [H][128][512] and scales [H][4]."""
+    H = w_uv.shape[1]
+    codes = torch.empty((H, 128, 512), dtype=torch.uint8, device=w_uv.device)
+    scales = torch.empty((H, 4), dtype=torch.float32, device=w_uv.device)
+    _check(_lib.mla_quantize_w_uv_fp8(_ptr(w_uv), H, _ptr(codes), _ptr(scales), _stream(stream)),
+           "mla_quantize_w_uv_fp8")
+    return Fp8Weight(codes, scales)
+
+
+def quantize_rows_fp8(x: torch.Tensor, stream=None):
+    """bf16 [..., cols] -> (codes uint8 [..., cols], scales fp32 [..., cols / 128])."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(tuple(x.shape[:-1]) + (cols // 128,), dtype=torch.float32, device=x.device)
+    _check(_lib.mla_quantize_rows_fp8(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _stream(stream)),
+           "mla_quantize_rows_fp8")
+    return codes, scales
+
+
+def absorb_q_fp8(q_nope: torch.Tensor, w: Fp8Weight, out: torch.Tensor | None = None, stream=None):
+    N, H, _ = q_nope.shape
+    if out is None:
+        out = torch.empty((N, H, 512), dtype=torch.bfloat16, device=q_nope.device)
+    _check(_lib.mla_absorb_q_fp8(_ptr(q_nope), _ptr(w.codes), _ptr(w.scales), _ptr(out), N, H, _stream(stream)),
+           "mla_absorb_q_fp8")
+    return out
+
+
+def out_uv_fp8(o_lat: torch.Tensor, w: Fp8Weight, out: torch.Tensor | None = None, stream=None):
+    N, H, _ = o_lat.shape
+    if out is None:
+        out = torch.empty((N, H, 128), dtype=torch.bfloat16, device=o_lat.device)
+    _check(_lib.mla_out_uv_fp8(_ptr(o_lat), _ptr(w.codes), _ptr(w.scales), _ptr(out), N, H, _stream(stream)),
+           "mla_out_uv_fp8")
+    return out
+
+
 def decode_attn(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_dev, num_clusters,
                 o_part, lse_part, o_lat, lse_out=None, status=None, stream=None):
     _check(_lib.mla_decode_attn(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(kv_pool),
@@ -214,15 +277,30 @@ class Decoder:
         self.lse = torch.empty((self.N, n_heads), dtype=torch.float32, device=dev)
         self.out = torch.empty((self.N, n_heads, 128), dtype=torch.bfloat16, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.fp8_uk: Fp8Weight | None = None
+        self.fp8_uv: Fp8Weight | None = None
+
+    def use_fp8_projections(self, w_uk, w_uv, stream=None):
+        """Run the two projections as FP8 block-quantised BMMs from now on:
+        W_UK and W_UV are quantised once here (their bf16 copies passed to
+        run() are then not read)."""
+        self.fp8_uk = quantize_w_uk_fp8(w_uk, stream)
+        self.fp8_uv = quantize_w_uv_fp8(w_uv, stream)
 
     def run(self, q_nope, q_rope, kv_pool, block_table, w_uk, w_uv, stream=None) -> DecodeOutputs:
-        absorb_q(q_nope, w_uk, self.q_lat, stream)
+        if self.fp8_uk is not None:
+            absorb_q_fp8(q_nope, self.fp8_uk, self.q_lat, stream)
+        else:
+            absorb_q(q_nope, w_uk, self.q_lat, stream)
         decode_attn(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev,
                     self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
                     self.lse, self.status, stream)
         if self.num_slots > 0:
             combine(self.dims, self.plan_dev, self.o_part, self.lse_part, self.o_lat, self.lse, stream)
-        out_uv(self.o_lat, w_uv, self.out, stream)
+        if self.fp8_uv is not None:
+            out_uv_fp8(self.o_lat, self.fp8_uv, self.out, stream)
+        else:
+            out_uv(self.o_lat, w_uv, self.out, stream)
         return DecodeOutputs(self.out, self.q_lat, self.o_lat, self.lse, self.status)
 
     @property

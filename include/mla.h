@@ -104,6 +104,45 @@ mla_status_t mla_out_uv(const void* o_lat, const void* w_uv, void* out,
                         int32_t n_tokens, int32_t n_heads, void* stream);
 
 /*
+ * FP8 block-quantised projections ("Lower latency and higher throughput with
+ * multi-node DeepSeek deployment", sections "Quantization" and "MLA layer":
+ * k_b_proj and v_b_proj as FP8 block-quantised BMMs).  Weights are quantised
+ * once, with one fp32 scale per 128 x 128 block of each head's matrix;
+ * activations are quantised on the fly inside the BMMs, with one scale per
+ * 128-element vector along K.  The format is E4M3 (largest finite 448).  A
+ * block's scale is s = amax / 448 (s = 1 for an all-zero block) and a value's
+ * code is E4M3(x * (448 / amax)), rounded to nearest even and saturated.  Each
+ * K-block's code products are summed in fp32 by the tensor cores, then
+ * scaled by s_act * s_weight; the outputs are bf16 (RNE).
+ *
+ * mla_quantize_w_uk_fp8: w_uk bf16 [512][n_heads][128] (read) ->
+ *   w_codes E4M3 [n_heads][512][128] (written; per head, rows k, K = d
+ *   contiguous) and w_scales fp32 [n_heads][4] (written; block k / 128).
+ * mla_quantize_w_uv_fp8: w_uv bf16 [512][n_heads][128] (read) ->
+ *   w_codes E4M3 [n_heads][128][512] (written; per head, rows v, K = k
+ *   contiguous) and w_scales fp32 [n_heads][4] (written; block k / 128).
+ * mla_quantize_rows_fp8: x bf16 [rows][cols] (cols a multiple of 128) ->
+ *   codes E4M3 [rows][cols] and scales fp32 [rows][cols / 128]: the same
+ *   per-vector quantisation the BMMs apply to their activations.
+ * mla_absorb_q_fp8: as mla_absorb_q, with the weight given as codes and
+ *   scales from mla_quantize_w_uk_fp8; q_nope is quantised per (token, head).
+ * mla_out_uv_fp8: as mla_out_uv, with codes and scales from
+ *   mla_quantize_w_uv_fp8; o_lat is quantised per (token, head, 128 columns).
+ * Codes are bytes; every pointer is a device pointer (16-byte aligned except
+ * the scale arrays, which need 4).  1 <= n_heads <= 128, 1 <= n_tokens <= 65536.
+ */
+mla_status_t mla_quantize_w_uk_fp8(const void* w_uk, int32_t n_heads, void* w_codes, float* w_scales,
+                                   void* stream);
+mla_status_t mla_quantize_w_uv_fp8(const void* w_uv, int32_t n_heads, void* w_codes, float* w_scales,
+                                   void* stream);
+mla_status_t mla_quantize_rows_fp8(const void* x, int64_t rows, int32_t cols, void* codes, float* scales,
+                                   void* stream);
+mla_status_t mla_absorb_q_fp8(const void* q_nope, const void* w_uk_codes, const float* w_uk_scales, void* q_lat,
+                              int32_t n_tokens, int32_t n_heads, void* stream);
+mla_status_t mla_out_uv_fp8(const void* o_lat, const void* w_uv_codes, const float* w_uv_scales, void* out,
+                            int32_t n_tokens, int32_t n_heads, void* stream);
+
+/*
  * Split-KV planning (host only, deterministic).  The decode kernel is a
  * persistent grid of 2-CTA clusters; each cluster walks a contiguous range of
  * the flattened (sequence, page) work list of one query position, so a long

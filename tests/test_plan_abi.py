@@ -165,3 +165,21 @@ def test_invalid_arguments_return_codes():
     small = (ctypes.c_int32 * 4)()
     assert lib.mla_plan(ctypes.byref(good), (ctypes.c_int32 * 2)(256, 256), 4, small, 16,
                         None) == mla.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_fp8_entry_points_validate_before_any_launch():
+    lib = mla._lib
+    assert lib.mla_quantize_w_uk_fp8(16, 0, 16, 16, None) == mla.MLA_ERR_UNSUPPORTED        # n_heads
+    assert lib.mla_quantize_w_uv_fp8(16, 129, 16, 16, None) == mla.MLA_ERR_UNSUPPORTED
+    assert lib.mla_quantize_w_uk_fp8(None, 8, 16, 16, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_quantize_w_uv_fp8(16, 8, 16, None, None) == mla.MLA_ERR_INVALID_ARG     # scales
+    assert b"w_scales" in lib.mla_last_error_string()
+    assert lib.mla_quantize_rows_fp8(16, 4, 100, 16, 16, None) == mla.MLA_ERR_UNSUPPORTED   # cols % 128
+    assert lib.mla_quantize_rows_fp8(16, -1, 128, 16, 16, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_quantize_rows_fp8(None, 0, 128, None, None, None) == mla.MLA_OK          # nothing to do
+    assert lib.mla_quantize_rows_fp8(24, 4, 128, 16, 16, None) == mla.MLA_ERR_INVALID_ARG   # misaligned x
+    assert lib.mla_absorb_q_fp8(16, 16, 16, 16, 0, 16, None) == mla.MLA_ERR_UNSUPPORTED     # n_tokens
+    assert lib.mla_absorb_q_fp8(16, 16, None, 16, 4, 16, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_out_uv_fp8(16, 24, 16, 16, 4, 16, None) == mla.MLA_ERR_INVALID_ARG       # misaligned codes
+    assert b"w_uv_codes" in lib.mla_last_error_string()
+    assert lib.mla_out_uv_fp8(16, 16, 16, 16, 4, 200, None) == mla.MLA_ERR_UNSUPPORTED      # n_heads
