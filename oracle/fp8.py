@@ -20,7 +20,7 @@ run as FP8 block-quantised BMMs.  In the absorbed decode path those are
 
 one (M, K) x (K, N) product per head h, with the tokens as M.
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * the FP8 format is E4M3 in its "FN" form: 4 exponent bits with bias 7, 3
     mantissa bits, no infinities, largest finite value 448, subnormals down
     to 2^-9;

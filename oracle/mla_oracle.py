@@ -25,7 +25,7 @@ inference cost computed?" (izhida.com, the expert answer): one RoPE'd key of
 width 64 shared by all heads, whose q.k score is *added* to the latent score.
 q_rope and k_rope arrive already rotated; no rotation happens here.
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * softmax scale = 1/sqrt(d_nope + d_rope) = 1/sqrt(192), no extra factor;
   * the softmax is the standard one over the key axis t;
   * the s new tokens are already in the cache: query i of s sits at position
