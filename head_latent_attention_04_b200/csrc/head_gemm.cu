@@ -24,6 +24,10 @@
 //   of up to 8 stages, each 16 KB of W_UV (MN-major: v contiguous) plus the
 //   tokens' 64-wide o_lat chunk.  The CTA prefetches its head's W_UV into L2
 //   before waiting for the merge kernel, so the weight read overlaps it.
+//
+// The same two products also run as FP8 (E4M3) block-quantised BMMs
+// (mla_absorb_q_fp8, mla_out_uv_fp8, with the weight and row quantisers), in
+// the section that follows the bf16 kernels.
 #include "mla_internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
