@@ -27,3 +27,11 @@ def test_algorithmic_accounting():
     # causal MTP: query i of a sequence of length T attends T - 1 + i keys
     acc2 = bench.algorithmic([10, 20], 2, 128)
     assert acc2["attn_flops"] == (9 + 10 + 19 + 20) * 2 * 128 * (2 * 512 + 64)
+
+
+def test_algorithmic_accounting_fp8_weights():
+    """E4M3 weights: one byte per element plus one fp32 scale per 128 x 128 block."""
+    bf = bench.algorithmic([4096] * 32, 1, 128)
+    f8 = bench.algorithmic([4096] * 32, 1, 128, weight_bytes=1)
+    assert bf["step_bytes"] - f8["step_bytes"] == 2 * 512 * 128 * 128 - 2 * 4 * 128 * 4
+    assert f8["attn_bytes"] == bf["attn_bytes"] and f8["step_flops"] == bf["step_flops"]
