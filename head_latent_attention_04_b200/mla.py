@@ -80,10 +80,17 @@ def _check(code: int, where: str):
 
 
 def _ptr(t) -> int | None:
+    """Device address of a tensor argument.  The library reads raw pointers,
+    so a host tensor (a host address handed to a kernel) or a strided view
+    (read as if contiguous) is refused here, before anything is launched."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor (the library assumes row-major layouts)")
     return t.data_ptr()
 
 
