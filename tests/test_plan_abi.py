@@ -183,3 +183,26 @@ def test_fp8_entry_points_validate_before_any_launch():
     assert lib.mla_out_uv_fp8(16, 24, 16, 16, 4, 16, None) == mla.MLA_ERR_INVALID_ARG       # misaligned codes
     assert b"w_uv_codes" in lib.mla_last_error_string()
     assert lib.mla_out_uv_fp8(16, 16, 16, 16, 4, 200, None) == mla.MLA_ERR_UNSUPPORTED      # n_heads
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """A host tensor would hand a host address to a kernel, and a strided view
+    would be read as if contiguous: both are refused before any CUDA call."""
+    import torch
+    q = torch.zeros((2, 4, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mla.absorb_q(q, torch.zeros((512, 4, 128), dtype=torch.bfloat16), torch.zeros((2, 4, 512), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mla.quantize_rows_fp8(torch.zeros((3, 128), dtype=torch.bfloat16))
+    # the contiguity check, seen without a GPU through a stand-in that claims to be on one
+    class FakeCuda:
+        is_cuda = True
+        def __init__(self, contiguous):
+            self.c = contiguous
+        def is_contiguous(self):
+            return self.c
+        def data_ptr(self):
+            return 4096
+    with pytest.raises(ValueError, match="contiguous"):
+        mla._ptr(FakeCuda(False))
+    assert mla._ptr(FakeCuda(True)) == 4096 and mla._ptr(None) is None and mla._ptr(16) == 16
