@@ -144,3 +144,23 @@ def out_uv_fp8(o_lat, Wq_uv, s_uv) -> np.ndarray:
     part = np.einsum("nhbk,hvbk->nhbv", oq.reshape(n, h, nkb, BLOCK), Wq)      # per K-block sums
     scale = so.astype(np.float64) * np.asarray(s_uv, dtype=np.float64)[None, :, :]   # [n][h][kb]
     return np.einsum("nhbv,nhb->nhv", part, scale)
+
+
+def quantize_cache(ckv) -> tuple:
+    """Latent cache rows c_KV [T][512] -> codes [T][512] and scales [T][4]: one
+    scale per 128-element block of each token's row, as for any activation
+    ("Quantization": activations carry a scale per 128-element vector).
+
+    Reading: only c_KV is quantised; the 64-wide k_rope part of a cache row
+    stays bf16 (the pages quantise GEMM operands by 128-blocks and say nothing
+    of the RoPE key, whose 128 bytes are a ninth of the row)."""
+    c = np.asarray(ckv, dtype=np.float32)
+    assert c.ndim == 2 and c.shape[1] % BLOCK == 0
+    return quantize_blocks(c, (1, BLOCK))
+
+
+def dequantize_cache(codes, scales) -> np.ndarray:
+    """codes [T][512] (values) and scales [T][4] -> float64 rows codes * scale."""
+    q = np.asarray(codes, dtype=np.float64)
+    s = np.repeat(np.asarray(scales, dtype=np.float64), BLOCK, axis=1)
+    return q * s

@@ -178,3 +178,47 @@ def test_fp8_bmm_error_against_bf16_path_is_quantisation_sized():
     rel = lambda a, b: np.linalg.norm(a - b) / np.linalg.norm(b)
     eq, eo = rel(F.absorb_fp8(q, Wq_uk, s_uk), ref_q), rel(F.out_uv_fp8(o, Wq_uv, s_uv), ref_o)
     assert 0.005 < eq < 0.06 and 0.005 < eo < 0.06, (eq, eo)
+
+
+def test_cache_quantisation_pins():
+    rng = np.random.default_rng(5)
+    # exact case: integers in [-7, 7] times a power of two per block, 7 * 2^j present
+    c = rng.integers(-7, 8, size=(9, 512)).astype(np.float64)
+    for t in range(9):
+        for kb in range(4):
+            j = int(rng.integers(-5, 3))
+            c[t, kb * 128:(kb + 1) * 128] *= 2.0 ** j
+            c[t, kb * 128 + 17] = -7 * 2.0 ** j
+    q, s = F.quantize_cache(c)
+    assert s.shape == (9, 4)
+    assert np.array_equal(F.dequantize_cache(q, s), c)
+    # general rows: within half a code spacing, scales from each block's own maximum
+    x = (rng.standard_normal((33, 512)) * 2.0).astype(np.float32)
+    q, s = F.quantize_cache(x)
+    for t in (0, 7, 32):
+        for kb in range(4):
+            blk = x[t, kb * 128:(kb + 1) * 128]
+            assert s[t, kb] == np.float32(np.float32(np.max(np.abs(blk))) / np.float32(448.0))
+    err = np.abs(F.dequantize_cache(q, s) - x)
+    assert np.all(err <= np.abs(x) * 2.0 ** -4 * (1 + 1e-6) + np.repeat(s, 128, axis=1) * 2.0 ** -10)
+
+
+def test_attention_over_an_exactly_quantised_cache_is_unchanged():
+    """Decode attention over the dequantised cache equals attention over the
+    original rows when the quantisation is exact: the cache quantiser changes
+    nothing but the stored bytes."""
+    rng = np.random.default_rng(6)
+    H, T = 4, 70
+    W_UK = rng.standard_normal((512, H, 128)) / np.sqrt(512)
+    W_UV = rng.standard_normal((512, H, 128)) / np.sqrt(512)
+    c = rng.integers(-7, 8, size=(T, 512)).astype(np.float64) * 2.0 ** -3
+    c[:, ::128] = 7 * 2.0 ** -3                            # every block holds its scale's maximum
+    k_rope = rng.standard_normal((T, 64))
+    q_nope = rng.standard_normal((1, H, 128))
+    q_rope = rng.standard_normal((1, H, 64))
+    codes, s = F.quantize_cache(c)
+    row = lambda ckv: np.concatenate([ckv, k_rope], axis=1)
+    a = O.mla_decode(q_nope, q_rope, [row(c)], W_UK, W_UV, 1, with_intermediates=False)["out"]
+    b = O.mla_decode(q_nope, q_rope, [row(F.dequantize_cache(codes, s))], W_UK, W_UV, 1,
+                     with_intermediates=False)["out"]
+    assert np.array_equal(a, b)
