@@ -3,9 +3,12 @@
 
 A step is the whole decode path on one batch: mla_absorb_q -> mla_decode_attn
 -> mla_combine -> mla_out_uv, with inputs resident in HBM.  The default
-workload is the DeepSeek-V2-shaped decode batch (B=32 sequences x 1 query
-token, 128 heads, T=4096 keys each, 64-token pages in a random permutation of
-the pool).  Prints ONE JSON line (rank 0).
+workload is the largest of the decode configurations that fits one GPU, the
+multi-token-prediction batch "mtp2": B=128 sequences x 2 causal query tokens,
+128 heads, T lognormal (median 4096, sigma 1, capped at 32768), 64-token pages
+in a random permutation of the pool, about 1 GB of latent cache.  --config
+selects the others (tiny, v2_4k, varlen, long128k).  Prints ONE JSON line
+(rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
@@ -44,8 +47,7 @@ sys.path.insert(0, ROOT)
 METRIC = "MLA decode tokens/s and effective cache TB/s (% of B200 roofline)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
-DECODE_SOURCES = ("head_latent_attention_04_b200/csrc/decode_attn.cu",
-                  "head_latent_attention_04_b200/csrc/ptx.cuh")
+DECODE_SOURCES = ("head_latent_attention_04_b200/csrc/decode_attn.cu",)
 
 
 def parse_args(argv=None):
@@ -53,7 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="v2_4k",
+    ap.add_argument("--config", default="mtp2",
                     choices=["tiny", "v2_4k", "varlen", "long128k", "mtp2"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of a CUDA graph")

@@ -283,6 +283,8 @@ mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void*
 
 size_t mla_noalloc_scratch_bytes(void) { return noalloc_scratch_bytes(); }
 
+void mla_set_wait_limit_ns(int64_t ns) { set_decode_wait_limit_ns(ns); }
+
 mla_status_t mla_debug_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
                                     int32_t n_pages, int32_t max_blocks_per_seq, int32_t num_blocks,
                                     void* out, int32_t* status, void* stream) {

@@ -118,8 +118,16 @@ mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_
                             const float* o_part, const float* lse_part, void* o_lat,
                             float* lse_out, void* stream) {
   // Column groups per thread: the smallest G with n_rows x 32 / G blocks within
-  // about one wave (2 blocks of 512 threads per SM on 148 SMs).
-  const long long wave = 2LL * 148;
+  // about one wave (2 blocks of 512 threads per SM).
+  static const int sms = [] {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = 148;
+    }
+    return n;
+  }();
+  const long long wave = 2LL * sms;
   int G = 1;
   while (G < 4 && (long long)n_rows * (32 / G) > wave) G *= 2;
   dim3 grid(n_rows, 32 / G);

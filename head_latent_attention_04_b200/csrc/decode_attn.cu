@@ -28,15 +28,17 @@
 // QK).  Shared memory holds five 36 KB stages of cache rows and one fp16 score
 // tile each way (own, peer); both tiles are read right after they land.
 //
-// Warp roles (480 threads): warp 0 TMA producer; warp 1 QK issuer and TMEM
+// Warp roles (512 threads): warp 0 TMA producer; warp 1 QK issuer and TMEM
 // owner; warp 2 PV issuer (two issuing threads, so a page waiting for its
 // softmax never holds back the next QK, and the tensor pipe takes work from
 // both); warps 3-6 score sender and q_lat loader (one thread per row);
 // warps 7-14 softmax / correction / epilogue (two warps per TMEM lane
-// quarter, one per 32-key half).  The grid
+// quarter, one per 32-key half); warp 15 copies each page's score tile to
+// the peer (one thread), so no sender waits on a copy.  The grid
 // is persistent: one cluster per SM pair, each walking the (row, page range)
-// items the host plan gives it.  Every wait is bounded (ptx::kWaitLimitNs);
-// on expiry the CTA sets MLA_STATUS_TIMEOUT and unwinds without trapping.
+// items the host plan gives it.  Every wait is bounded (200 ms by default,
+// mla_set_wait_limit_ns); on expiry the CTA sets MLA_STATUS_TIMEOUT, stops its
+// peer, drains the copies and products it issued and returns without trapping.
 #include "mla_internal.h"
 #include "plan_format.h"
 #include "ptx.cuh"
@@ -44,6 +46,8 @@
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
+
+#include <atomic>
 
 namespace mla {
 namespace {
@@ -66,8 +70,8 @@ constexpr int kOffPMax = kOffXOwn + kXBytes;                 // fp32 [2 pages][2
 constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;      // fp32 [2 items][2 halves][128] half-row sums
 constexpr int kOffBar = kOffLSum + 4 * kRows * 4;
 
-constexpr int kThreads = 480;            // 15 warps
-constexpr int kSenderWarp0 = 3, kSoftWarp0 = 7;
+constexpr int kThreads = 512;            // 16 warps
+constexpr int kSoftWarp0 = 7, kCopyWarp = 15;   // senders are warps 3 .. 6
 constexpr int kSoftWarps = 8;
 
 constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemQR = 480, kTmemCols = 512;
@@ -87,6 +91,7 @@ struct DecodeParams {
   int32_t* status;
   int n_heads, max_blocks, num_blocks, s_q, causal, B, n_rows, num_clusters;
   float scale_log2;             // scale * log2(e)
+  uint64_t wait_ns;             // limit of every protocol wait (drains of issued work use the default)
 };
 
 struct Bars {
@@ -104,20 +109,60 @@ struct Bars {
   uint64_t o_free, qk_done, pv_done;
   uint64_t pmax[2][4];   // the two softmax warps of row quarter q posted their page-b half-row maxima
   uint64_t lsum[4];      // the two softmax warps of row quarter q posted their half-row sums (per item)
+  uint32_t tmem_base;    // TMEM allocation
+  uint32_t sent_count;   // score tiles this CTA has copied to its peer
+  WaitCtl wc;            // abort flag and wait limit of every role
 };
-constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 16 + 1024;
+constexpr int kSmemBytes = kOffBar + (int)sizeof(Bars) + 1024;
 
 __device__ __forceinline__ void report(int32_t* status, int bits) {
   if (status) atomicOr(status, bits);
 }
 
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile WaitCtl* wc) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
 }
-// For data a peer CTA wrote with st.async: its complete_tx releases at cluster
-// scope, so the waiter must acquire at cluster scope to see the stores.
-__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, abort));
+// For data the peer CTA's bulk copy wrote: its complete_tx releases at cluster
+// scope, so the waiter must acquire at cluster scope to see the bytes.
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile WaitCtl* wc) {
+  return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, wc));
+}
+
+// The plan fixes each row's key count (kv_len) from the host seq_lens it was
+// made with.  True if the device seq_lens (T of the item's sequence) now give
+// another count: the softmax then masks every key of the item, so the row is
+// written as zeros with LSE -inf, and MLA_STATUS_BAD_SEQLEN is reported.
+__device__ __forceinline__ bool item_stale(const int32_t* w, int T, const DecodeParams& p) {
+  const int want = p.causal ? T - p.s_q + 1 + w[kItQi] : T;
+  return want != w[kItKvLen];
+}
+
+// Keys of the item's last page that are attended (1 .. 64).  When fewer than
+// 64, that page is loaded shifted: its first `attended` keys land in stage
+// rows [64 - attended, 64) and the rows above them are the TMA's zero fill
+// (a negative row coordinate), so no stale or non-finite cache row past the
+// key count ever reaches the P.c_KV product (where 0 * Inf would be NaN).
+__device__ __forceinline__ int last_page_keys(const int32_t* w) {
+  return w[kItKvLen] - (w[kItPageEnd] - 1) * kPage;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two fp16 pairs -> their element-wise sums in fp32: lo = a.lo + b.lo, hi =
+// a.hi + b.hi, each operand taken exactly and the sum rounded once to fp32
+// (the mixed-precision add takes one fp16 operand as is).
+__device__ __forceinline__ void add_f16x2_to_f32(uint32_t a, uint32_t b, float& lo, float& hi) {
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t.reg .f32 t0, t1;\n\t"
+      "mov.b32 {a0, a1}, %2;\n\tmov.b32 {b0, b1}, %3;\n\t"
+      "cvt.f32.f16 t0, b0;\n\tcvt.f32.f16 t1, b1;\n\t"
+      "add.rn.f32.f16 %0, a0, t0;\n\tadd.rn.f32.f16 %1, a1, t1;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(a), "r"(b));
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -137,14 +182,21 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   float* s_pmax = reinterpret_cast<float*>(smem + kOffPMax);
   float* s_lsum = reinterpret_cast<float*>(smem + kOffLSum);
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + sizeof(Bars));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* tmem_slot = &bars->tmem_base;
+  volatile WaitCtl* wc = &bars->wc;
+  volatile uint32_t* sent_count = &bars->sent_count;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
   const int cid = (int)cluster_id_x();
+  // A role that gives up stops both CTAs of the pair (the peer would otherwise
+  // wait for score tiles that never come): it raises its own flag and the
+  // peer's, so after the final cluster barrier both flags tell the same story.
+  auto give_up = [&]() {
+    wc->abort = 1;
+    st_cluster_u32(mapa(smem_u32((const void*)&wc->abort), peer), 1u);
+  };
 
-  // The plan must match the launch (uniform over the grid).
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -170,7 +222,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       mbar_init(&bars->pmax[1][q], 2);
       mbar_init(&bars->lsum[q], 2);
     }
-    *abort_flag = 0;
+    wc->abort = 0;
+    wc->limit_ns = p.wait_ns;
+    *sent_count = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_kv);
     prefetch_tmap(&tm_rope);
@@ -181,7 +235,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   }
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // peer barriers initialised before any remote arrive
+  cluster_sync();   // peer barriers and flags initialised before any remote access
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   griddep_wait();   // set-up above overlaps the previous kernel; global memory only from here
@@ -189,43 +243,49 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 
   // The section offsets follow from the cluster count, so the cluster's item
   // range is read without first waiting for the header (checked alongside).
+  // The plan must match the launch (uniform over the grid).
   const int32_t* plan = p.plan;
   const int off_cluster = kPlanHeaderWords, off_items = kPlanHeaderWords + p.num_clusters + 1;
   const int32_t* items = plan + off_items;
   const int it_begin_raw = plan[off_cluster + cid], it_end_raw = plan[off_cluster + cid + 1];
   const bool plan_ok = plan[kHdrMagic] == kPlanMagic && plan[kHdrNumClusters] == p.num_clusters &&
                        plan[kHdrNumRows] == p.n_rows && plan[kHdrHeads] == p.n_heads &&
+                       plan[kHdrB] == p.B && plan[kHdrSq] == p.s_q &&
+                       plan[kHdrMaxBlocks] == p.max_blocks && plan[kHdrCausal] == (p.causal ? 1 : 0) &&
                        plan[kHdrOffCluster] == off_cluster && plan[kHdrOffItems] == off_items;
   const int it_begin = plan_ok ? it_begin_raw : 0;
   const int it_end = plan_ok ? it_end_raw : 0;
-  if (!plan_ok && threadIdx.x == 0 && rank == 0 && cid == 0) report(p.status, MLA_STATUS_BAD_SEQLEN);
+  if (!plan_ok && threadIdx.x == 0 && rank == 0 && cid == 0) report(p.status, MLA_STATUS_BAD_PLAN);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // Lane 0 waits and issues; the whole warp fetches block ids 32 pages at a
     // time with one coalesced load, so a page's TMA never waits on its own
-    // block-table read.
+    // block-table read.  The first 32 ids of an item are read together with
+    // the item's sequence length, in one round trip.
     int g = 0;
     bool fail = false;
-    for (int it = it_begin; it < it_end && !fail && !*abort_flag; ++it) {
+    for (int it = it_begin; it < it_end && !fail; ++it) {
+      if (__any_sync(0xffffffffu, wc->abort != 0)) break;   // warp-uniform
       const int32_t* w = items + (size_t)it * kItemWords;
       const int b = w[kItB], pb = w[kItPageBegin], pe = w[kItPageEnd];
+      const int shift = kPage - min(last_page_keys(w), kPage);   // zero-filled rows of the last page
+      int my_blk = pb + lane < pe ? p.block_table[(size_t)b * p.max_blocks + pb + lane] : 0;
       if (lane == 0 && it + 1 < it_end) {   // the next item's query rows, so that its loaders read them from L2
         const size_t nrow = (size_t)items[(size_t)(it + 1) * kItemWords + kItRow];
         bulk_prefetch_l2(p.q_lat + nrow * p.n_heads * 512, (uint32_t)p.n_heads * 1024u);
         bulk_prefetch_l2(p.q_rope + nrow * p.n_heads * 64, (uint32_t)p.n_heads * 128u);
       }
-      int my_blk = 0;
       for (int pg = pb; pg < pe && !fail; ++pg, ++g) {
         const int rel = pg - pb;
-        if ((rel & 31) == 0) {
+        if ((rel & 31) == 0 && rel > 0) {
           const int q = pg + lane;
           my_blk = q < pe ? p.block_table[(size_t)b * p.max_blocks + q] : 0;
         }
         int blk = __shfl_sync(0xffffffffu, my_blk, rel & 31);
         if (lane == 0) {
           const int s = g % kStages;
-          if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, abort_flag)) {
+          if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, wc)) {
             fail = true;
           } else {
             if (blk < 0 || blk >= p.num_blocks) {
@@ -233,11 +293,12 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
               blk = 0;
             }
             uint8_t* st = s_kv + s * kStageBytes;
-            mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
+            const int y = pg + 1 == pe ? -shift : 0;   // first row of the block to load
+            mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);   // zero-filled bytes count too
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-              tma_load_2d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, blk * kPage);
-            tma_load_2d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, blk * kPage);
+              tma_load_3d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, y, blk);
+            tma_load_3d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, y, blk);
           }
         }
         fail = __shfl_sync(0xffffffffu, fail, 0);
@@ -246,19 +307,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     }
     if (lane == 0) {
       if (fail) {
-        *abort_flag = 1;
+        give_up();
         report(p.status, MLA_STATUS_TIMEOUT);
       }
       // every issued load must land before the CTA may exit
       for (int k = g - 1; k >= 0 && k >= g - kStages; --k)
-        mbar_wait(&bars->kv_full[k % kStages], (k / kStages) & 1, nullptr);
+        mbar_drain(&bars->kv_full[k % kStages], (k / kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
     // S = [q_lat | q_rope] . [c_KV | k_rope]^T over this CTA's 288 columns:
-    // M = 128 rows, N = 64 keys, 16 MMAs with A = q_lat from TMEM and 2 with
-    // A = q_rope from shared memory.  S is single-buffered; the sender frees
-    // it (s_read) as soon as it has copied the product out.
+    // M = 128 rows, N = 64 keys, 16 MMAs with A = q_lat and 2 with A = q_rope,
+    // both from TMEM.  S is single-buffered; the sender frees it (s_read) as
+    // soon as it has copied the product out.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
       const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
@@ -268,11 +329,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       for (int it = it_begin; ok && it < it_end; ++it) {
         const int32_t* w = items + (size_t)it * kItemWords;
         const int n = w[kItPageEnd] - w[kItPageBegin];
-        if (!mbar_wait(&bars->q_full, (it - it_begin) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&bars->q_full, (it - it_begin) & 1, wc)) { ok = false; break; }
         for (int j = 0; j < n; ++j, ++g) {
           const int s = g % kStages;
-          if (!mbar_wait(&bars->kv_full[s], (g / kStages) & 1, abort_flag) ||
-              (g > 0 && !mbar_wait(&bars->s_read, (g - 1) & 1, abort_flag))) {
+          if (!mbar_wait(&bars->kv_full[s], (g / kStages) & 1, wc) ||
+              (g > 0 && !mbar_wait(&bars->s_read, (g - 1) & 1, wc))) {
             ok = false;
             break;
           }
@@ -291,11 +352,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (ok) mma_commit(&bars->q_empty);   // q_lat and q_rope (TMEM) may be replaced
       }
       if (!ok) {
-        *abort_flag = 1;
+        give_up();
         report(p.status, MLA_STATUS_TIMEOUT);
       }
       mma_commit(&bars->qk_done);
-      mbar_wait(&bars->qk_done, 0, nullptr);   // no MMA may still write TMEM at dealloc
+      mbar_drain(&bars->qk_done, 0);   // no MMA may still write TMEM at dealloc
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ PV issuer
@@ -312,8 +373,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         const int ii = it - it_begin;
         for (int j = 0; j < n; ++j, ++g) {
           const int s = g % kStages;
-          if (!mbar_wait(&bars->p_full, g & 1, abort_flag) ||
-              (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, abort_flag))) {
+          if (!mbar_wait(&bars->p_full, g & 1, wc) ||
+              (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, wc))) {
             ok = false;
             break;
           }
@@ -331,11 +392,11 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (ok) mma_commit(&bars->o_done);
       }
       if (!ok) {
-        *abort_flag = 1;
+        give_up();
         report(p.status, MLA_STATUS_TIMEOUT);
       }
       mma_commit(&bars->pv_done);
-      mbar_wait(&bars->pv_done, 0, nullptr);
+      mbar_drain(&bars->pv_done, 0);
     }
   } else if (warp < kSoftWarp0) {
     // ------------------------------------------------------------ query loader and score sender (4 warps)
@@ -344,22 +405,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // previous item's last QK has completed; the producer has prefetched those
     // rows into L2.  Per page it reads this CTA's partial scores (its 288
     // columns) as soon as the QK product lands, frees S, rounds to fp16 into
-    // the own tile, and one thread pushes that tile to the peer's tile with a
+    // the own tile, and the copy warp pushes that tile to the peer's tile with a
     // bulk copy that completes on the peer's x_recv.  Thread = one row, 64
-    // keys; 16-byte chunks XOR-swizzled by (row & 7).  (Per-thread st.async
-    // stores into the peer raced with the peer's reads under load; the bulk
-    // copy is deterministic.)
+    // keys; 16-byte chunks XOR-swizzled by (row & 7).
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t x_peer = mapa(smem_u32(s_xpeer), peer);
-    const uint32_t x_recv_peer = mapa(smem_u32(&bars->x_recv), peer);
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
-      const int n = w[kItPageEnd] - w[kItPageBegin];
       const int ii = it - it_begin;
-      if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, abort_flag)) goto sender_fail;
+      if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, wc)) goto sender_fail;
       {
         const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)w[kItRow] * p.n_heads + r) * 512 +
                                                           256 * rank);
@@ -390,9 +446,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->q_full);
       }
+      const int n = w[kItPageEnd] - w[kItPageBegin];
       for (int j = 0; j < n; ++j, ++g) {
         uint32_t v[64];
-        if (!warp_wait(&bars->s_full, g & 1, abort_flag)) goto sender_fail;
+        if (!warp_wait(&bars->s_full, g & 1, wc)) goto sender_fail;
         tc_fence_after();
         tmem_ld32(tmem + lane_addr + kTmemS, *reinterpret_cast<uint32_t(*)[32]>(v));
         tmem_ld32(tmem + lane_addr + kTmemS + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
@@ -404,7 +461,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 #pragma unroll
         for (int k = 0; k < 32; ++k) hv[k] = pack_f16(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
         // single tile: page g - 1's own tile must have been read by the softmax and the copy
-        if (g >= 1 && !warp_wait(&bars->own_free, (g - 1) & 1, abort_flag)) goto sender_fail;
+        if (g >= 1 && !warp_wait(&bars->own_free, (g - 1) & 1, wc)) goto sender_fail;
         {
           uint8_t* own = s_xown + r * kXRow;
 #pragma unroll
@@ -412,28 +469,50 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             *reinterpret_cast<uint4*>(own + ((k ^ (r & 7)) << 4)) =
                 make_uint4(hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
         }
-        fence_proxy_async_smem();   // the bulk copy below reads the tile through the async proxy
+        fence_proxy_async_smem();   // the copy warp's bulk copy reads the tile through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->own_full);
-        if (warp == kSenderWarp0 && lane == 0) {
-          // one bulk copy of the whole tile to the peer, completing on its x_recv;
-          // the local tile may be rewritten only after the copy has read it
-          // and the peer must have read page g - 1 out of its peer tile
-          if (!mbar_wait(&bars->own_full, g & 1, abort_flag) ||
-              (g >= 1 && !mbar_wait(&bars->x_sendok, (g - 1) & 1, abort_flag)))
-            goto sender_fail;
-          bulk_copy_to_peer(x_peer, smem_u32(s_xown), kXBytes, x_recv_peer);
-          bulk_commit();
-          bulk_wait_read<0>();
-          mbar_arrive(&bars->own_free);
-        }
       }
     }
     goto sender_done;
   sender_fail:
-    *abort_flag = 1;
+    give_up();
     if (lane == 0) report(p.status, MLA_STATUS_TIMEOUT);
   sender_done:;
+  } else if (warp == kCopyWarp) {
+    // ------------------------------------------------------------ score copy (one thread)
+    // Per page: one bulk copy of the own fp16 tile to the peer's tile,
+    // completing on the peer's x_recv, once the 4 sender warps have written
+    // it and the peer has read page g - 1 out of its tile.  The own tile may
+    // be rewritten once the copy has read it (own_free).  A warp of its own,
+    // so that waiting for the copy never holds back the next page's score read.
+    if (lane == 0) {
+      const uint32_t x_peer = mapa(smem_u32(s_xpeer), peer);
+      const uint32_t x_recv_peer = mapa(smem_u32(&bars->x_recv), peer);
+      uint32_t sent = 0;
+      bool ok = true;
+      int g = 0;
+      for (int it = it_begin; ok && it < it_end; ++it) {
+        const int32_t* w = items + (size_t)it * kItemWords;
+        const int n = w[kItPageEnd] - w[kItPageBegin];
+        for (int j = 0; j < n; ++j, ++g) {
+          if (!mbar_wait(&bars->own_full, g & 1, wc) ||
+              (g >= 1 && !mbar_wait(&bars->x_sendok, (g - 1) & 1, wc))) {
+            ok = false;
+            break;
+          }
+          bulk_copy_to_peer(x_peer, smem_u32(s_xown), kXBytes, x_recv_peer);
+          bulk_commit();
+          *sent_count = ++sent;
+          bulk_wait_read<0>();
+          mbar_arrive(&bars->own_free);
+        }
+      }
+      if (!ok) {
+        give_up();
+        report(p.status, MLA_STATUS_TIMEOUT);
+      }
+    }
   } else {
     // ------------------------------------------------------------ softmax / epilogue (8 warps)
     // Thread = (row r, key half c): keys [32c, 32c+32) of each page, output
@@ -441,15 +520,25 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int quarter = warp & 3;
     const int c = (warp - kSoftWarp0) >> 2;
     const int r = quarter * 32 + lane;
+    const int tid = threadIdx.x - kSoftWarp0 * 32;    // 0 .. 255
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     const uint32_t x_sendok_peer = mapa(smem_u32(&bars->x_sendok), peer);
+    bool out_of_range = false;   // a fp16 partial overflowed: a reference max of +Inf, or a NaN sum
+    // The sequence length of the next item is loaded one item ahead, so that
+    // the stale-plan check never waits for memory at an item boundary.
+    int T_next = it_begin < it_end ? p.seq_lens[items[(size_t)it_begin * kItemWords + kItB]] : 0;
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
-      const int row = w[kItRow], pb = w[kItPageBegin], n = w[kItPageEnd] - pb, slot = w[kItSlot];
-      const int kv_len = w[kItKvLen];
+      const int row = w[kItRow], slot = w[kItSlot];
+      const int n = w[kItPageEnd] - w[kItPageBegin];
       const int ii = it - it_begin;
+      const bool stale = item_stale(w, T_next, p);
+      if (it + 1 < it_end) T_next = p.seq_lens[items[(size_t)(it + 1) * kItemWords + kItB]];
+      if (stale && tid == 0 && rank == 0) report(p.status, MLA_STATUS_BAD_SEQLEN);
+      // keys masked in the item's last page: the zero-filled rows of its shifted load
+      const int shift_last = kPage - min(last_page_keys(w), kPage);
 
       float m_ref = -CUDART_INF_F, l_run = 0.f;
       for (int j = 0; j < n; ++j) {
@@ -457,32 +546,28 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         // full score = fp16(own partial) + fp16(peer partial), identical in both CTAs.
         // The own tile is read (and released) first: it lands before the peer's.
         uint4 po[4], pr[4];
-        uint32_t used = 0;
         const uint32_t off_base = (uint32_t)(4 * c);
-        if (!warp_wait(&bars->own_full, gj & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait(&bars->own_full, gj & 1, wc)) goto softmax_fail;
         {
           const uint8_t* orow = s_xown + r * kXRow;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 4; ++k)
             po[k] = *reinterpret_cast<const uint4*>(orow + (((off_base + k) ^ (r & 7)) << 4));
-            used |= po[k].x ^ po[k].w;
-          }
           uint32_t bar_addr = smem_u32(&bars->own_free);
-          asm volatile("" : "+r"(bar_addr) : "r"(used));   // arrive only after the own tile was read
+          // arrive only after the own tile was read (one word of each 16-byte load)
+          asm volatile("" : "+r"(bar_addr) : "r"(po[0].x ^ po[1].x ^ po[2].x ^ po[3].x));
           __syncwarp();
           if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_addr) : "memory");
         }
-        if (!warp_wait_cluster(&bars->x_recv, gj & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait_cluster(&bars->x_recv, gj & 1, wc)) goto softmax_fail;
         {
           const uint8_t* xrow = s_xpeer + r * kXRow;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int k = 0; k < 4; ++k)
             pr[k] = *reinterpret_cast<const uint4*>(xrow + (((off_base + k) ^ (r & 7)) << 4));
-            used |= pr[k].x ^ pr[k].w;
-          }
           // the peer tile is consumed: re-arm x_recv for page gj + 1, then let the peer refill it
           uint32_t ok_addr = x_sendok_peer;
-          asm volatile("" : "+r"(ok_addr) : "r"(used));   // issue only after the tile was read
+          asm volatile("" : "+r"(ok_addr) : "r"(pr[0].x ^ pr[1].x ^ pr[2].x ^ pr[3].x));
           __syncwarp();
           if (lane == 0) {
             if (warp == kSoftWarp0) mbar_arrive_expect_tx(&bars->x_recv, kXBytes);
@@ -494,34 +579,31 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           const uint32_t* ow = reinterpret_cast<const uint32_t*>(po);
           const uint32_t* pw = reinterpret_cast<const uint32_t*>(pr);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float2 a = unpack_f16x2(ow[k]);
-            const float2 o = unpack_f16x2(pw[k]);
-            sc[2 * k] = a.x + o.x;
-            sc[2 * k + 1] = a.y + o.y;
-          }
+          for (int k = 0; k < 16; ++k) add_f16x2_to_f32(ow[k], pw[k], sc[2 * k], sc[2 * k + 1]);
         }
-        const int tok0 = (pb + j) * kPage + 32 * c;
-        if (tok0 + 32 > kv_len) {
+        // masked columns [0, lo) of this page: the last page's zero fill, or all
+        // of them when the device seq_lens disagree with the plan
+        const int lo = stale ? kPage : (j == n - 1 ? shift_last : 0);
+        if (lo > 32 * c) {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
-            if (tok0 + k >= kv_len) sc[k] = -CUDART_INF_F;
+            if (32 * c + k < lo) sc[k] = -CUDART_INF_F;
         }
         float mloc;
         {
-          float t[16];
+          float t[11], u[4];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) t[k] = fmaxf(sc[k], sc[k + 16]);
+          for (int k = 0; k < 10; ++k) t[k] = fmax3(sc[3 * k], sc[3 * k + 1], sc[3 * k + 2]);
+          t[10] = fmaxf(sc[30], sc[31]);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) t[k] = fmaxf(t[k], t[k + 8]);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) t[k] = fmaxf(t[k], t[k + 4]);
-          mloc = fmaxf(fmaxf(t[0], t[2]), fmaxf(t[1], t[3]));
+          for (int k = 0; k < 3; ++k) u[k] = fmax3(t[3 * k], t[3 * k + 1], t[3 * k + 2]);
+          u[3] = fmaxf(t[9], t[10]);
+          mloc = fmaxf(fmax3(u[0], u[1], u[2]), u[3]);
         }
         s_pmax[(b * 2 + c) * kRows + r] = mloc;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->pmax[b][quarter]);
-        if (!warp_wait(&bars->pmax[b][quarter], (gj >> 1) & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait(&bars->pmax[b][quarter], (gj >> 1) & 1, wc)) goto softmax_fail;
         const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kRows + r]) * sl2;
 
         // lazy reference max (log2 domain): move it only when the row max grows by > 2^8
@@ -546,9 +628,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
         // the single P buffer is free once the previous page's PV product has completed
-        if (gj >= 1 && !warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
+        if (gj >= 1 && !warp_wait(&bars->o_full, (gj - 1) & 1, wc)) goto softmax_fail;
         if (__any_sync(0xffffffffu, move && j > 0)) {
-          if (!warp_wait(&bars->o_full, (gj - 1) & 1, abort_flag)) goto softmax_fail;
           tc_fence_after();
           const float a = (move && j > 0) ? alpha : 1.f;
 #pragma unroll 1
@@ -569,16 +650,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (lane == 0) mbar_arrive(&bars->p_full);
       }
 
-      // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot
+      // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot.  A
+      // stale item has P = 0 throughout: its row is written as zeros.
+      out_of_range |= (m_ref == CUDART_INF_F) | (l_run != l_run);
       {
-        if (!warp_wait(&bars->o_done, ii & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait(&bars->o_done, ii & 1, wc)) goto softmax_fail;
         tc_fence_after();
         float* ls = s_lsum + (ii & 1) * 2 * kRows;    // [item parity][half][row]
         ls[c * kRows + r] = l_run;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->lsum[quarter]);
-        if (!warp_wait(&bars->lsum[quarter], ii & 1, abort_flag)) goto softmax_fail;
+        if (!warp_wait(&bars->lsum[quarter], ii & 1, wc)) goto softmax_fail;
         l_run = ls[r] + ls[kRows + r];             // same order in both halves
+        out_of_range |= (l_run != l_run);
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const bool valid = r < p.n_heads;
         const bool o_lat_32b = (reinterpret_cast<uintptr_t>(p.o_lat) & 31) == 0;
@@ -625,9 +709,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     }
     goto softmax_done;
   softmax_fail:
-    *abort_flag = 1;
+    give_up();
     if (lane == 0) report(p.status, MLA_STATUS_TIMEOUT);
-  softmax_done:;
+  softmax_done:
+    if (__any_sync(0xffffffffu, out_of_range) && lane == 0 && rank == 0) report(p.status, MLA_STATUS_SCORE_RANGE);
   }
 
   tc_fence_before();
@@ -636,7 +721,28 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
   __syncwarp();
   cluster_sync();   // no CTA leaves while its peer may still write into its shared memory
+  // After a give-up, roles may have left their loops with the peer's last
+  // score tile still on its way here.  A give-up raises both CTAs' flags
+  // before its CTA reaches the barrier above, so after it both flags agree
+  // and both CTAs take the same branch.  A copy is only sent after the
+  // receiver consumed the previous one, so at most the peer's last copy is
+  // outstanding: wait (default limit) for its phase, which lands because it
+  // was issued, then meet the peer once more.
+  {
+    // (addresses recomputed here rather than kept live through the roles)
+    Bars* b = reinterpret_cast<Bars*>(((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023)) + kOffBar);
+    if (*reinterpret_cast<volatile int*>(&b->wc.abort) != 0) {
+      if (threadIdx.x == 0) {
+        const uint32_t sent_by_peer = ld_cluster_u32(mapa(smem_u32(&b->sent_count), cluster_ctarank() ^ 1u));
+        if (sent_by_peer > 0) mbar_drain<true>(&b->x_recv, (sent_by_peer - 1) & 1);
+      }
+      __syncwarp();
+      cluster_sync();
+    }
+  }
 }
+
+std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
 
 // Set once per process, so that later launches can be captured in a CUDA graph.
 cudaError_t decode_smem_attr() {
@@ -652,14 +758,16 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
                                 const int32_t* seq_lens, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream) {
+  // The pool as (column, row within the block, block): a box may start at a
+  // negative row, which the TMA fills with zeros (the shifted last page).
   CUtensorMap tm_kv, tm_rope;
-  const uint64_t pdims[2] = {576, (uint64_t)d.num_blocks * kPage};
-  const uint64_t pstr[1] = {576 * 2};
-  const uint32_t box_kv[2] = {64, kPage};
-  const uint32_t box_rope[2] = {32, kPage};
-  mla_status_t st = encode_tmap_bf16(&tm_kv, kv_pool, 2, pdims, pstr, box_kv, CU_TENSOR_MAP_SWIZZLE_128B);
+  const uint64_t pdims[3] = {576, (uint64_t)kPage, (uint64_t)d.num_blocks};
+  const uint64_t pstr[2] = {576 * 2, (uint64_t)kPage * 576 * 2};
+  const uint32_t box_kv[3] = {64, kPage, 1};
+  const uint32_t box_rope[3] = {32, kPage, 1};
+  mla_status_t st = encode_tmap_bf16(&tm_kv, kv_pool, 3, pdims, pstr, box_kv, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != MLA_OK) return st;
-  st = encode_tmap_bf16(&tm_rope, kv_pool, 2, pdims, pstr, box_rope, CU_TENSOR_MAP_SWIZZLE_64B);
+  st = encode_tmap_bf16(&tm_rope, kv_pool, 3, pdims, pstr, box_rope, CU_TENSOR_MAP_SWIZZLE_64B);
   if (st != MLA_OK) return st;
   const int N = d.B * d.s_q;
 
@@ -683,6 +791,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
   p.n_rows = N;
   p.num_clusters = num_clusters;
   p.scale_log2 = d.scale * 1.4426950408889634f;
+  p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
 
   cudaError_t e = decode_smem_attr();
   if (e == cudaSuccess) {
@@ -691,6 +800,10 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return MLA_OK;
+}
+
+void set_decode_wait_limit_ns(int64_t ns) {
+  g_wait_limit_ns.store(ns > 0 ? (uint64_t)ns : kWaitLimitNs, std::memory_order_relaxed);
 }
 
 mla_status_t decode_max_clusters(int32_t* n) {

@@ -689,10 +689,7 @@ mla_status_t launch_absorb_q(const void* q_nope, const void* w_uk, void* q_lat, 
   // shared memory: 1 KB alignment slack + weight tile + token chunks (the output
   // tile reuses them) + barriers, padded so that at most 512 / cols CTAs share an
   // SM and their TMEM allocations always fit together
-  int smem = 1024 + 2 * kATileBytes + 2 * bn * 128 + 64;
-  const int ctas_per_sm = 512 / (int)tmem_cols_for(bn);
-  const int floor_bytes = kSmemPerSM / (ctas_per_sm + 1) - 1024 + 1;
-  if (smem < floor_bytes) smem = floor_bytes;
+  const int smem = pad_smem_for_tmem(1024 + 2 * kATileBytes + 2 * bn * 128 + 64, (int)tmem_cols_for(bn));
   GemmParams p{n_tokens, n_heads, bn, 0};
   cudaError_t e = set_smem_attrs();
   if (e == cudaSuccess) {

@@ -61,6 +61,7 @@ mla_status_t launch_gather_pages(const void* kv_pool, const int32_t* block_table
                                  int32_t n_pages, int32_t max_blocks, int32_t num_blocks, void* out,
                                  int32_t* status, void* stream);
 mla_status_t decode_max_clusters(int32_t* n);
+void set_decode_wait_limit_ns(int64_t ns);
 mla_status_t decode_attn_combine_noalloc(const mla_dims_t& d, const void* q_lat, const void* q_rope,
                                          const void* kv_pool, const int32_t* block_table,
                                          const int32_t* seq_lens, const void* plan_host,

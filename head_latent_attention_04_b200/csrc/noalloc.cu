@@ -15,6 +15,10 @@
 // real address up with cudaGetSymbolAddress, with that device current, and
 // caches it.  Make that first call before any stream capture.
 //
+// The plan is copied into the array with cudaMemcpyAsync on the caller's
+// stream; from pinned host memory that copy may still be reading plan_host
+// after the call returns.
+//
 // All calls share the one array, which keeps whatever the last call left in
 // it.  Nothing in it needs to start at zero: the attention kernel writes every
 // partial slot the plan uses before the merge reads it.  Calls whose work can
@@ -40,10 +44,17 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
-mla_status_t scratch_for_current_device(void** out) {
+// The array of the current device, which must also be the device of `stream`
+// (the plan copy and both kernels run there).
+mla_status_t scratch_for_current_device(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  int stream_dev = dev;
+  e = cudaStreamGetDevice(stream, &stream_dev);
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "cudaStreamGetDevice: %s", cudaGetErrorString(e));
+  if (stream_dev != dev)
+    return set_error(MLA_ERR_INVALID_ARG, "stream belongs to device %d but device %d is current", stream_dev, dev);
   if (dev < 0 || dev >= kMaxDevices) return set_error(MLA_ERR_UNSUPPORTED, "device index %d too large", dev);
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_ptr[dev]) {
@@ -71,9 +82,14 @@ mla_status_t decode_attn_combine_noalloc(const mla_dims_t& d, const void* q_lat,
   const int32_t* plan = static_cast<const int32_t*>(plan_host);
   if (plan_bytes < kPlanHeaderWords * 4 || plan[kHdrMagic] != kPlanMagic)
     return set_error(MLA_ERR_INVALID_ARG, "plan_host is not a plan made by mla_plan");
-  if (plan[kHdrNumClusters] != num_clusters || plan[kHdrNumRows] != d.B * d.s_q || plan[kHdrHeads] != d.n_heads)
+  if (plan[kHdrNumClusters] != num_clusters || plan[kHdrB] != d.B || plan[kHdrSq] != d.s_q ||
+      plan[kHdrNumRows] != d.B * d.s_q || plan[kHdrHeads] != d.n_heads ||
+      plan[kHdrMaxBlocks] != d.max_blocks_per_seq || plan[kHdrCausal] != (d.causal ? 1 : 0))
     return set_error(MLA_ERR_INVALID_ARG, "plan was made for other dims or another cluster count");
-  const size_t words = (size_t)plan[kHdrTotalWords];
+  const int64_t words_signed = plan[kHdrTotalWords];
+  if (words_signed < kPlanHeaderWords || plan[kHdrNumSlots] < 0)
+    return set_error(MLA_ERR_INVALID_ARG, "plan_host is not a plan made by mla_plan");
+  const size_t words = (size_t)words_signed;
   if (words * 4 > plan_bytes) return set_error(MLA_ERR_INVALID_ARG, "plan_bytes smaller than the plan");
   const size_t slots = (size_t)plan[kHdrNumSlots];
   const size_t plan_region = round_up(words * 4, 256);
@@ -86,15 +102,15 @@ mla_status_t decode_attn_combine_noalloc(const mla_dims_t& d, const void* q_lat,
                      "(use mla_decode_attn + mla_combine with caller workspace, or fewer clusters)",
                      need, kScratchBytes);
 
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* base = nullptr;
-  mla_status_t st = scratch_for_current_device(&base);
+  mla_status_t st = scratch_for_current_device(s, &base);
   if (st != MLA_OK) return st;
   unsigned char* b = static_cast<unsigned char*>(base);
   int32_t* plan_dev = reinterpret_cast<int32_t*>(b);
   float* lse_part = reinterpret_cast<float*>(b + plan_region);
   float* o_part = reinterpret_cast<float*>(b + plan_region + lse_region);
 
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(plan_dev, plan_host, words * 4, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "plan copy: %s", cudaGetErrorString(e));
   st = launch_decode_attn(d, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_dev, num_clusters, o_part,

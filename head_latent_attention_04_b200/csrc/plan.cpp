@@ -108,6 +108,8 @@ mla_status_t build_plan(const mla_dims_t& d, const int32_t* seq_lens, int32_t nu
   plan[kHdrOffItems] = off_items;
   plan[kHdrOffRows] = off_rows;
   plan[kHdrTotalWords] = total;
+  plan[kHdrMaxBlocks] = d.max_blocks_per_seq;
+  plan[kHdrCausal] = d.causal ? 1 : 0;
 
   int32_t* cl = plan + off_cluster;
   for (int32_t c = 0; c <= num_clusters; ++c) cl[c] = 0;

@@ -28,6 +28,8 @@ enum PlanHeader : int {
   kHdrOffItems = 9,     // items[num_items][kItemWords]
   kHdrOffRows = 10,     // row_slot_begin[num_rows + 1]
   kHdrTotalWords = 11,
+  kHdrMaxBlocks = 12,   // columns of block_table the plan was made for
+  kHdrCausal = 13,      // the dims' causal flag the plan was made with
 };
 
 // One work item: a contiguous page range of one query row's key sequence.

@@ -44,12 +44,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
-// Arrive (release at cluster scope) on a barrier given by its shared::cluster address.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-
 // Relaxed arrive on a barrier given by its shared::cluster address: a signal
 // with no memory ordering (the caller orders its own accesses beforehand).
 __device__ __forceinline__ void mbar_arrive_relaxed_cluster(uint32_t cluster_addr) {
@@ -62,19 +56,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Non-blocking test of the phase of parity `parity`.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -96,10 +77,14 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_
 }
 
 // Bounded wait for the phase of parity `parity` to complete.  Returns false if
-// the time limit passed or *abort became non-zero (another role gave up).
-// abort == nullptr: only the time limit ends the wait (used to drain copies).
+// `limit_ns` of global time passed or *abort became non-zero (another role
+// gave up); both are checked after every 16 unsuccessful polls, so that a
+// spinning warp takes few issue slots from the warps doing the work.
+// abort == nullptr: only the time limit ends the wait (used to drain copies
+// and tensor-core work already issued, which complete on their own).
 template <bool kClusterAcquire = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (kClusterAcquire ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity))
     return true;
   const uint64_t t0 = globaltimer();
@@ -108,9 +93,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return true;
     if ((i & 15) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
     }
   }
+}
+
+// Abort flag and time limit of a CTA's waits, kept in shared memory so that a
+// waiting thread holds one 32-bit address instead of both in registers.
+struct WaitCtl {
+  int abort;                   // non-zero: another role (or the peer CTA) gave up
+  int pad;
+  unsigned long long limit_ns; // bound of each wait
+};
+
+// mbar_wait with the abort flag and the limit read from `ctl` on the slow path.
+template <bool kClusterAcquire = false>
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile WaitCtl* ctl) {
+  if (kClusterAcquire ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity))
+    return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (kClusterAcquire ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity))
+      return true;
+    if ((i & 15) == 0) {
+      if (ctl->abort) return false;
+      if (globaltimer() - t0 > ctl->limit_ns) return false;
+    }
+  }
+}
+
+// Wait, with the default limit and no abort flag, for work that was already
+// issued and completes on its own (copies, tensor-core products).
+template <bool kClusterAcquire = false>
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  return mbar_wait<kClusterAcquire>(bar, parity, static_cast<volatile int*>(nullptr));
 }
 
 // ---------------------------------------------------------------- programmatic dependent launch
@@ -150,18 +166,14 @@ __device__ __forceinline__ uint32_t mapa(uint32_t smem_addr, uint32_t rank) {
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, float b, float c,
-                                              float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
+// 32-bit load / store of a word in a cluster peer's shared memory (relaxed).
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
 }
-
-__device__ __forceinline__ void st_cluster_v4u(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c,
-                                               uint32_t d) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "r"(a), "r"(b),
-               "r"(c), "r"(d)
-               : "memory");
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 
 // 32-byte global store of eight words (address 32-byte aligned).
@@ -184,22 +196,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
-}
-
-// Streaming variant: the cache lines read are marked evict-first in L2.
-__device__ __forceinline__ void tma_load_2d_stream(void* dst, const CUtensorMap* m, uint64_t* bar,
-                                                   int x, int y, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int x,
@@ -230,7 +226,6 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
       "r"(src_smem), "r"(bytes), "r"(bar_cluster)
       : "memory");
 }
-// Hint: bring [gptr, gptr + bytes) into L2 (16-byte aligned, multiple of 16 bytes), in 16 KB pieces.
 // L2 prefetch of one tensor-map box (a hint: no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int x, int y, int z) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(reinterpret_cast<uint64_t>(m)),
@@ -238,6 +233,7 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int x, 
                : "memory");
 }
 
+// Hint: bring [gptr, gptr + bytes) into L2 (16-byte aligned, multiple of 16 bytes), in 16 KB pieces.
 __device__ __forceinline__ void bulk_prefetch_l2(const void* gptr, uint32_t bytes) {
   const char* c = static_cast<const char*>(gptr);
   for (uint32_t off = 0; off < bytes; off += 16384u) {
@@ -256,10 +252,6 @@ __device__ __forceinline__ void bulk_wait_read() {
 template <int N>
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // Generic-proxy writes to shared memory -> visible to the async proxy (TMA, tcgen05).
@@ -427,8 +419,6 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_f16x2(uint32_t u) {
   return __half22float2(*reinterpret_cast<__half2*>(&u));
 }
-// The value a float pair takes after a round trip through fp16.
-__device__ __forceinline__ float2 round_f16x2(float lo, float hi) { return unpack_f16x2(pack_f16(lo, hi)); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;   // low 16 bits = lo, high 16 bits = hi, each rounded to nearest even

@@ -23,12 +23,12 @@ _lib = ctypes.CDLL(_LIB_PATH)
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED = 0, 1, 2
 MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_TIMEOUT = 3, 4, 5
-STATUS_BAD_BLOCK, STATUS_TIMEOUT, STATUS_BAD_SEQLEN = 0x1, 0x2, 0x4
+STATUS_BAD_BLOCK, STATUS_TIMEOUT, STATUS_BAD_SEQLEN, STATUS_BAD_PLAN, STATUS_SCORE_RANGE = 0x1, 0x2, 0x4, 0x8, 0x10
 EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
            "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes",
            "mla_quantize_w_uk_fp8", "mla_quantize_w_uv_fp8", "mla_quantize_rows_fp8", "mla_absorb_q_fp8",
-           "mla_out_uv_fp8")
+           "mla_out_uv_fp8", "mla_set_wait_limit_ns")
 
 
 class MlaDims(ctypes.Structure):
@@ -65,6 +65,8 @@ for _name, _args in {
 
 _lib.mla_noalloc_scratch_bytes.argtypes = []
 _lib.mla_noalloc_scratch_bytes.restype = _sz
+_lib.mla_set_wait_limit_ns.argtypes = [ctypes.c_int64]
+_lib.mla_set_wait_limit_ns.restype = None
 
 
 class MlaError(RuntimeError):
@@ -109,6 +111,13 @@ def make_dims(B, s_q, n_heads, max_blocks, num_blocks, scale=None, causal=True) 
         scale = 1.0 / math.sqrt(128 + 64)
     return MlaDims(B, s_q, n_heads, 128, 64, 512, 128, 64, max_blocks, num_blocks, float(scale),
                    1 if causal else 0)
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound on each pipeline wait of decode launches made from now on
+    (process-wide; 0 restores the 200 ms default).  A wait past it makes the
+    kernel give up cleanly with STATUS_TIMEOUT."""
+    _lib.mla_set_wait_limit_ns(int(ns))
 
 
 def max_clusters() -> int:

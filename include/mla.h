@@ -58,7 +58,11 @@ typedef enum {
 /* Bits set in the device status word. */
 #define MLA_STATUS_BAD_BLOCK   0x1   /* block_table entry outside [0, num_blocks): block 0 used */
 #define MLA_STATUS_TIMEOUT     0x2   /* a bounded device wait expired; outputs are invalid */
-#define MLA_STATUS_BAD_SEQLEN  0x4   /* device seq_lens disagree with the plan */
+#define MLA_STATUS_BAD_SEQLEN  0x4   /* a row's device seq_lens disagrees with the plan: row skipped */
+#define MLA_STATUS_BAD_PLAN    0x8   /* the plan was made for other dims or another cluster count:
+                                        nothing computed */
+#define MLA_STATUS_SCORE_RANGE 0x10  /* a partial score of an attended key left the fp16 range
+                                        (|x| > 65504) or was not a number: outputs are invalid */
 
 /* Problem dimensions of one decode batch. */
 typedef struct {
@@ -175,7 +179,12 @@ mla_status_t mla_plan(const mla_dims_t* dims, const int32_t* seq_lens_host, int3
  *   q_rope       bf16 [N][n_heads][64]      (post-rotation)
  *   kv_pool      bf16 [num_blocks][64][576] (token row = c_KV (512) | k_rope (64))
  *   block_table  int32 [B][max_blocks_per_seq]
- *   seq_lens     int32 [B]  T_b, counting the s_q new tokens (checked against the plan)
+ *   seq_lens     int32 [B]  T_b, counting the s_q new tokens.  A plan is valid for the
+ *                lengths it was made from: the kernel compares each row's key count
+ *                with these device values, and a row that disagrees is skipped
+ *                (written as zeros with LSE -inf) and MLA_STATUS_BAD_SEQLEN is
+ *                set.  A decode loop whose lengths grow every step makes a new
+ *                plan (mla_plan, host only, microseconds) and copies it each step.
  *   plan_dev     the plan from mla_plan, copied to the device
  *   num_clusters the num_clusters the plan was built for (grid = 2 * num_clusters CTAs)
  *   o_part       fp32, slots x n_heads x 512  workspace (split rows); element
@@ -186,6 +195,12 @@ mla_status_t mla_plan(const mla_dims_t* dims, const int32_t* seq_lens_host, int3
  *   lse_out      fp32 [N][n_heads] or NULL    natural-log LSE of the scaled logits
  *   status       int32 [1] or NULL
  * Rows that the plan splits are completed by mla_combine.
+ *
+ * Numerics: the two CTAs of a cluster each score half of the 576 columns and
+ * exchange their partial scores rounded to fp16; a partial of an attended key
+ * beyond the fp16 range sets MLA_STATUS_SCORE_RANGE.  Cache rows past a row's
+ * key count (page tails, other queries' keys) may hold anything, NaN and Inf
+ * included: the kernel zeroes them in shared memory before the P.c_KV product.
  */
 mla_status_t mla_decode_attn(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
                              const void* kv_pool, const int32_t* block_table,
@@ -223,7 +238,16 @@ mla_status_t mla_combine(const mla_dims_t* dims, const void* plan_dev, const flo
  *   - it allocates nothing and frees nothing;
  *   - all calls share the array, and it keeps the last call's contents
  *     (nothing in it needs to start at zero); calls that overlap on the GPU
- *     race on it, so serialise them.
+ *     race on it, so serialise them;
+ *   - the plan is copied to the array with cudaMemcpyAsync on `stream`: from
+ *     pageable memory the call returns once the bytes are staged, but from
+ *     pinned memory the copy may still be reading plan_host after the call
+ *     returns, so do not overwrite it until the stream has passed this call;
+ *   - `stream` must belong to the current device (MLA_ERR_INVALID_ARG
+ *     otherwise): the array used is the current device's.
+ * The plan is checked against dims and num_clusters on the host before any
+ * copy (magic word, cluster count, B, s_q, n_heads, max_blocks_per_seq,
+ * causal, and that plan_bytes covers it); a mismatch is MLA_ERR_INVALID_ARG.
  * The other arguments mean what they mean for mla_decode_attn / mla_combine;
  * o_lat (and lse_out if non-NULL) receive the finished rows.
  */
@@ -236,6 +260,18 @@ mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void*
 
 /* Size in bytes of the device array mla_decode_attn_combine_noalloc works in. */
 size_t mla_noalloc_scratch_bytes(void);
+
+/*
+ * mla_set_wait_limit_ns -- upper bound, in nanoseconds of GPU global time, on
+ * each wait of the decode kernel's pipeline roles for every decode launch
+ * made after the call (process-wide).  Default 200 ms; ns <= 0 restores it.
+ * When a wait runs past the bound the kernel sets MLA_STATUS_TIMEOUT, stops
+ * both CTAs of the cluster, waits (with the default bound) for the copies and
+ * tensor-core products it has already issued, frees its tensor memory and
+ * returns; the context stays usable.  A tiny bound makes the time-out path run
+ * on purpose, which is what the failure-detection test does.
+ */
+void mla_set_wait_limit_ns(int64_t ns);
 
 /*
  * mla_debug_gather_pages -- copies the cache rows of sequence b, in token

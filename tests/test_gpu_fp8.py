@@ -1,15 +1,16 @@
 """FP8 block-quantised projections on the GPU against the FP8 oracle.
 
 The quantisers are compared code by code and scale by scale (a float32
-decision on both sides); the BMMs within the rel-Frobenius tolerance of the
-bf16 path, against the oracle's float64 product of the oracle's own codes."""
+decision on both sides); the BMMs within the tolerance of the bf16 path
+(relative Frobenius <= 5e-3 and max abs <= 2e-2), against the oracle's
+float64 product of the oracle's own codes."""
 import numpy as np
 import pytest
 import torch
 
 from head_latent_attention_04_b200 import workloads as W
 from oracle import fp8 as F
-from tests.gpu_helpers import rel_fro
+from tests.gpu_helpers import check_out, rel_fro
 
 pytestmark = pytest.mark.gpu
 
@@ -70,7 +71,7 @@ def test_absorb_q_fp8_matches_oracle(mla, N, H):
     torch.cuda.synchronize()
     codes, s = F.quantize_w_uk(wuk.float().numpy())
     want = F.absorb_fp8(q.float().numpy(), codes, s)
-    assert rel_fro(got.float().cpu().numpy(), want) < 5e-3
+    check_out(got, want)
 
 
 @pytest.mark.parametrize("N,H", [(1, 1), (2, 16), (37, 128), (128, 128), (130, 3), (300, 7)])
@@ -84,7 +85,7 @@ def test_out_uv_fp8_matches_oracle(mla, N, H):
     torch.cuda.synchronize()
     codes, s = F.quantize_w_uv(wuv.float().numpy())
     want = F.out_uv_fp8(o.float().numpy(), codes, s)
-    assert rel_fro(got.float().cpu().numpy(), want) < 5e-3
+    check_out(got, want)
 
 
 @pytest.mark.parametrize("N,H", [(37, 128), (300, 5)])
@@ -101,8 +102,8 @@ def test_fp8_projections_write_only_their_rows(mla, N, H):
     assert bool((big_q[N:] == 3.0).all()) and bool((big_o[N:] == 3.0).all())
     ck, sk = F.quantize_w_uk(wuk.float().numpy())
     cv, sv = F.quantize_w_uv(wuv.float().numpy())
-    assert rel_fro(big_q[:N].float().cpu().numpy(), F.absorb_fp8(q.float().cpu().numpy(), ck, sk)) < 5e-3
-    assert rel_fro(big_o[:N].float().cpu().numpy(), F.out_uv_fp8(o.float().cpu().numpy(), cv, sv)) < 5e-3
+    check_out(big_q[:N], F.absorb_fp8(q.float().cpu().numpy(), ck, sk))
+    check_out(big_o[:N], F.out_uv_fp8(o.float().cpu().numpy(), cv, sv))
 
 
 def test_fp8_step_against_bf16_step(mla):
@@ -121,4 +122,4 @@ def test_fp8_step_against_bf16_step(mla):
     assert 1e-3 < err < 0.08, err
     codes, s = F.quantize_w_uk(w.w_uk.float().cpu().numpy())
     want_q = F.absorb_fp8(w.q_nope.float().cpu().numpy(), codes, s)
-    assert rel_fro(got.q_lat.float().cpu().numpy(), want_q) < 5e-3
+    check_out(got.q_lat, want_q)

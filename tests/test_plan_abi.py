@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def test_library_exports_every_declared_symbol():
     header = open(os.path.join(ROOT, "include", "mla.h")).read()
-    declared = set(re.findall(r"^\s*(?:mla_status_t|int32_t|size_t|const char\*)\s+(mla_\w+)\s*\(", header, re.M))
+    declared = set(re.findall(r"^\s*(?:mla_status_t|int32_t|size_t|void|const char\*)\s+(mla_\w+)\s*\(", header, re.M))
     assert declared == set(mla.EXPORTS)
     lib = ctypes.CDLL(mla._LIB_PATH)
     for name in declared:
@@ -165,6 +165,51 @@ def test_invalid_arguments_return_codes():
     small = (ctypes.c_int32 * 4)()
     assert lib.mla_plan(ctypes.byref(good), (ctypes.c_int32 * 2)(256, 256), 4, small, 16,
                         None) == mla.MLA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_plan_header_records_the_dims():
+    """Header words 12 and 13 hold max_blocks_per_seq and the causal flag, which
+    the kernel and the allocation-free entry point check besides B, s_q, h."""
+    d = mla.make_dims(3, 2, 64, 17, 100, causal=True)
+    buf, _ = mla.plan(d, [5, 700, 1000], 6)
+    assert buf[5] == 64 and buf[6] == 2 and buf[7] == 3 and buf[12] == 17 and buf[13] == 1
+    buf, _ = mla.plan(mla.make_dims(3, 1, 64, 17, 100, causal=False), [5, 700, 1000], 6)
+    assert buf[13] == 0
+
+
+def _noalloc(dims, plan, nbytes, clusters):
+    """The allocation-free entry point with stand-in device pointers: every case
+    below must be refused on the host, before any CUDA call."""
+    return mla._lib.mla_decode_attn_combine_noalloc(ctypes.byref(dims), 16, 16, 16, 16, 16, plan.ctypes.data,
+                                                    nbytes, clusters, 16, None, None, None)
+
+
+def test_noalloc_refuses_plans_that_do_not_match():
+    dims = mla.make_dims(4, 1, 128, 64, 1000)
+    plan, _ = mla.plan(dims, [4096, 100, 3000, 64], 8)
+    bad = plan.copy()
+    bad[0] = 0                                                   # magic word
+    assert _noalloc(dims, bad, bad.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
+    assert b"not a plan" in mla._lib.mla_last_error_string()
+    assert _noalloc(dims, plan, plan.nbytes, 9) == mla.MLA_ERR_INVALID_ARG      # cluster count
+    assert _noalloc(dims, plan, 4 * (int(plan[11]) - 1), 8) == mla.MLA_ERR_INVALID_ARG   # truncated
+    assert b"plan_bytes" in mla._lib.mla_last_error_string()
+    assert _noalloc(dims, plan, 60, 8) == mla.MLA_ERR_INVALID_ARG              # not even a header
+    bad = plan.copy()
+    bad[11] = -5                                                 # negative length
+    assert _noalloc(dims, bad, bad.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
+    # same number of rows (B * s_q = 4), other B and s_q
+    d22 = mla.make_dims(2, 2, 128, 64, 1000)
+    p22, _ = mla.plan(d22, [4096, 100], 8)
+    assert _noalloc(dims, p22, p22.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
+    assert _noalloc(d22, plan, plan.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
+    # a plan made for a wider block table, for the other causal flag, or for other heads
+    wider, _ = mla.plan(mla.make_dims(4, 1, 128, 80, 1000), [4096, 100, 3000, 64], 8)
+    assert _noalloc(dims, wider, wider.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
+    nc, _ = mla.plan(mla.make_dims(4, 1, 128, 64, 1000, causal=False), [4096, 100, 3000, 64], 8)
+    assert _noalloc(dims, nc, nc.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
+    other_h, _ = mla.plan(mla.make_dims(4, 1, 64, 64, 1000), [4096, 100, 3000, 64], 8)
+    assert _noalloc(dims, other_h, other_h.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
 
 
 def test_fp8_entry_points_validate_before_any_launch():
