@@ -16,17 +16,20 @@
 // two CTAs splits the latent dimension: CTA r owns latent columns
 // [256r, 256r + 256) and RoPE columns [32r, 32r + 32).  Each CTA stages only
 // its half of every cache row (each byte is read from HBM once) and computes
-// a partial score over its 288 columns.  The partial scores are rounded to
-// fp16 and exchanged through distributed shared memory (one bulk copy per page,
-// counted on the receiver's mbarrier); both CTAs then form fp16(S0) + fp16(S1) in fp32,
+// a partial score over its 288 columns.  The partial scores, scaled to log2
+// units (scale * log2(e)), are rounded to fp16 and exchanged through
+// distributed shared memory (one bulk copy per page, counted on the
+// receiver's mbarrier); both CTAs then add fp16(S0) + fp16(S1) as fp16 pairs,
 // which is bit-identical in the pair, so both take the same softmax
 // decisions.  Each CTA accumulates its 256 output columns.
 //
 // TMEM (512 columns): O [0,256) fp32, S [256,320) fp32 (released as soon as
-// the sender has read it), P [320,352) bf16 (A operand of the PV product),
-// q_lat half [352,480) and q_rope half [480,496) as bf16 pairs (A operands of
-// QK).  Shared memory holds five 36 KB stages of cache rows and one fp16 score
-// tile each way (own, peer); both tiles are read right after they land.
+// the sender has read it), two P buffers [320,352) and [352,384) bf16 (A
+// operand of the PV product; page g uses buffer g & 1, so the softmax of a
+// page never waits for the previous page's PV product), q_lat half [384,512)
+// as bf16 pairs (A operand of QK).  Shared memory holds five 36 KB stages of
+// cache rows, one fp16 score tile each way (own, peer), both read right after
+// they land, and the q_rope half (A operand of the two RoPE MMAs).
 //
 // Warp roles (512 threads): warp 0 TMA producer; warp 1 QK issuer and TMEM
 // owner; warp 2 PV issuer (two issuing threads, so a page waiting for its
@@ -67,14 +70,15 @@ constexpr int kOffKV = 0;
 constexpr int kOffXPeer = kOffKV + kStages * kStageBytes;   // peer's partial scores (one tile)
 constexpr int kOffXOwn = kOffXPeer + kXBytes;                // own partial scores (fp16, one tile)
 constexpr int kOffPMax = kOffXOwn + kXBytes;                 // fp32 [2 pages][2 halves][128] half-row maxima
-constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;      // fp32 [2 items][2 halves][128] half-row sums
-constexpr int kOffBar = kOffLSum + 4 * kRows * 4;
+constexpr int kOffLSum = kOffPMax + 4 * kRows * 4;     // fp32 [2 items][2 halves][128] half-row sums
+constexpr int kOffQRope = kOffLSum + 4 * kRows * 4;    // bf16 q_rope half, 128 rows x 64 B (SW64, A of QK)
+constexpr int kOffBar = kOffQRope + kRows * 64;
 
 constexpr int kThreads = 512;            // 16 warps
 constexpr int kSoftWarp0 = 7, kCopyWarp = 15;   // senders are warps 3 .. 6
 constexpr int kSoftWarps = 8;
 
-constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 352, kTmemQR = 480, kTmemCols = 512;
+constexpr uint32_t kTmemO = 0, kTmemS = 256, kTmemP = 320, kTmemQ = 384, kTmemCols = 512;   // P: two 32-column buffers
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale O only when the max grows by > 2^8
 
@@ -104,7 +108,7 @@ struct Bars {
   uint64_t x_recv;       // peer's fp16 partial scores landed in the peer tile (1 arrival + 16 KB tx)
   uint64_t x_sendok;     // peer has read its peer tile, which this CTA may refill (8 remote arrivals)
   uint64_t p_full;       // P written (O rescaled if needed), 8 softmax warps
-  uint64_t o_full;        // PV product of a page complete (awaited one page behind, for rescaling)
+  uint64_t o_full[2];     // PV product of a page complete, per P buffer (page g uses buffer g & 1)
   uint64_t o_done;        // every PV product of the current item complete (epilogue)
   uint64_t o_free, qk_done, pv_done;
   uint64_t pmax[2][4];   // the two softmax warps of row quarter q posted their page-b half-row maxima
@@ -119,13 +123,16 @@ __device__ __forceinline__ void report(int32_t* status, int bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Suspend-time hint of the pipeline waits (0: no hint, spin).
+constexpr uint32_t kWaitHintNs = 0;
+
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile WaitCtl* wc) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, wc));
+  return __all_sync(0xffffffffu, mbar_wait<false, kWaitHintNs>(bar, parity, wc));
 }
 // For data the peer CTA's bulk copy wrote: its complete_tx releases at cluster
 // scope, so the waiter must acquire at cluster scope to see the bytes.
 __device__ __forceinline__ bool warp_wait_cluster(uint64_t* bar, uint32_t parity, volatile WaitCtl* wc) {
-  return __all_sync(0xffffffffu, mbar_wait<true>(bar, parity, wc));
+  return __all_sync(0xffffffffu, mbar_wait<true, kWaitHintNs>(bar, parity, wc));
 }
 
 // The plan fixes each row's key count (kv_len) from the host seq_lens it was
@@ -146,23 +153,26 @@ __device__ __forceinline__ int last_page_keys(const int32_t* w) {
   return w[kItKvLen] - (w[kItPageEnd] - 1) * kPage;
 }
 
-// Three-input maximum (one instruction on sm_100).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+// fp16 pair sum and maximum (round to nearest even; the maximum of -inf and x is x).
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t hmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
-// Two fp16 pairs -> their element-wise sums in fp32: lo = a.lo + b.lo, hi =
-// a.hi + b.hi, each operand taken exactly and the sum rounded once to fp32
-// (the mixed-precision add takes one fp16 operand as is).
-__device__ __forceinline__ void add_f16x2_to_f32(uint32_t a, uint32_t b, float& lo, float& hi) {
-  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\t.reg .f32 t0, t1;\n\t"
-      "mov.b32 {a0, a1}, %2;\n\tmov.b32 {b0, b1}, %3;\n\t"
-      "cvt.f32.f16 t0, b0;\n\tcvt.f32.f16 t1, b1;\n\t"
-      "add.rn.f32.f16 %0, a0, t0;\n\tadd.rn.f32.f16 %1, a1, t1;\n\t}"
+// (a.lo + c, a.hi + c) in fp32 for an fp16 pair a: the mixed-precision add
+// takes the fp16 operand exactly and rounds the sum once.
+__device__ __forceinline__ void add_f16x2_to_f32(uint32_t a, float c, float& lo, float& hi) {
+  asm("{\n\t.reg .f16 a0, a1;\n\t"
+      "mov.b32 {a0, a1}, %2;\n\t"
+      "add.rn.f32.f16 %0, a0, %3;\n\tadd.rn.f32.f16 %1, a1, %3;\n\t}"
       : "=f"(lo), "=f"(hi)
-      : "r"(a), "r"(b));
+      : "r"(a), "f"(c));
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -181,6 +191,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
   uint8_t* s_xown = smem + kOffXOwn;
   float* s_pmax = reinterpret_cast<float*>(smem + kOffPMax);
   float* s_lsum = reinterpret_cast<float*>(smem + kOffLSum);
+  uint8_t* s_qrope = smem + kOffQRope;
   Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
   uint32_t* tmem_slot = &bars->tmem_base;
   volatile WaitCtl* wc = &bars->wc;
@@ -212,7 +223,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     mbar_init(&bars->x_sendok, kSoftWarps);
     mbar_init(&bars->p_full, kSoftWarps);
     mbar_arrive_expect_tx(&bars->x_recv, kXBytes);   // armed for page 0
-    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->o_full[0], 1);
+    mbar_init(&bars->o_full[1], 1);
     mbar_init(&bars->o_done, 1);
     mbar_init(&bars->o_free, kSoftWarps);
     mbar_init(&bars->qk_done, 1);
@@ -261,8 +273,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // ------------------------------------------------------------ TMA producer
     // Lane 0 waits and issues; the whole warp fetches block ids 32 pages at a
     // time with one coalesced load, so a page's TMA never waits on its own
-    // block-table read.  The first 32 ids of an item are read together with
-    // the item's sequence length, in one round trip.
+    // block-table read.  (An L2 prefetch of the blocks a few pages ahead was
+    // measured slower at distances 2 to 12.)
     int g = 0;
     bool fail = false;
     for (int it = it_begin; it < it_end && !fail; ++it) {
@@ -285,7 +297,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         int blk = __shfl_sync(0xffffffffu, my_blk, rel & 31);
         if (lane == 0) {
           const int s = g % kStages;
-          if (g >= kStages && !mbar_wait(&bars->kv_empty[s], ((g / kStages) - 1) & 1, wc)) {
+          if (g >= kStages && !mbar_wait<false, kWaitHintNs>(&bars->kv_empty[s], ((g / kStages) - 1) & 1, wc)) {
             fail = true;
           } else {
             if (blk < 0 || blk >= p.num_blocks) {
@@ -319,85 +331,86 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // S = [q_lat | q_rope] . [c_KV | k_rope]^T over this CTA's 288 columns:
     // M = 128 rows, N = 64 keys, 16 MMAs with A = q_lat and 2 with A = q_rope,
     // both from TMEM.  S is single-buffered; the sender frees it (s_read) as
-    // soon as it has copied the product out.
-    if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
-      const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
-      const uint64_t kr_desc0 = sdesc(smem_u32(s_kv) + 4 * kChunkBytes, 16, 512, kSwizzle64B);
-      bool ok = true;
-      int g = 0;
-      for (int it = it_begin; ok && it < it_end; ++it) {
-        const int32_t* w = items + (size_t)it * kItemWords;
-        const int n = w[kItPageEnd] - w[kItPageBegin];
-        if (!mbar_wait(&bars->q_full, (it - it_begin) & 1, wc)) { ok = false; break; }
-        for (int j = 0; j < n; ++j, ++g) {
-          const int s = g % kStages;
-          if (!mbar_wait(&bars->kv_full[s], (g / kStages) & 1, wc) ||
-              (g > 0 && !mbar_wait(&bars->s_read, (g - 1) & 1, wc))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t kvd = kv_desc0 + (uint64_t)((s * kStageBytes) >> 4);
-          const uint64_t krd = kr_desc0 + (uint64_t)((s * kStageBytes) >> 4);
-#pragma unroll
-          for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16, A = q_lat from TMEM
-            mma_ts(tmem + kTmemS, tmem + kTmemQ + 8 * t,
-                   kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
-#pragma unroll
-          for (int t = 0; t < 2; ++t)    // RoPE half: K = 32, A = q_rope from TMEM
-            mma_ts(tmem + kTmemS, tmem + kTmemQR + 8 * t, krd + (uint64_t)(t * 2), idesc_qk, 1);
-          mma_commit(&bars->s_full);
+    // soon as it has copied the product out.  The whole warp runs the loop
+    // (descriptors stay warp-uniform) and one elected lane issues.
+    const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
+    const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
+    const uint64_t kr_desc0 = sdesc(smem_u32(s_kv) + 4 * kChunkBytes, 16, 512, kSwizzle64B);
+    const uint64_t qr_desc = sdesc(smem_u32(s_qrope), 16, 512, kSwizzle64B);
+    bool ok = true;
+    int g = 0;
+    for (int it = it_begin; ok && it < it_end; ++it) {
+      const int32_t* w = items + (size_t)it * kItemWords;
+      const int n = w[kItPageEnd] - w[kItPageBegin];
+      if (!warp_wait(&bars->q_full, (it - it_begin) & 1, wc)) { ok = false; break; }
+      for (int j = 0; j < n; ++j, ++g) {
+        const int s = g % kStages;
+        if (!warp_wait(&bars->kv_full[s], (g / kStages) & 1, wc) ||
+            (g > 0 && !warp_wait(&bars->s_read, (g - 1) & 1, wc))) {
+          ok = false;
+          break;
         }
-        if (ok) mma_commit(&bars->q_empty);   // q_lat and q_rope (TMEM) may be replaced
+        tc_fence_after();
+        const uint64_t kvd = kv_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+        const uint64_t krd = kr_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+#pragma unroll
+        for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16, A = q_lat from TMEM
+          mma_ts_elect(tmem + kTmemS, tmem + kTmemQ + 8 * t,
+                       kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)    // RoPE half: K = 32, A = q_rope from shared memory
+          mma_ss_elect(tmem + kTmemS, qr_desc + (uint64_t)(t * 2), krd + (uint64_t)(t * 2), idesc_qk, 1);
+        mma_commit_elect(&bars->s_full);
       }
-      if (!ok) {
-        give_up();
-        report(p.status, MLA_STATUS_TIMEOUT);
-      }
-      mma_commit(&bars->qk_done);
-      mbar_drain(&bars->qk_done, 0);   // no MMA may still write TMEM at dealloc
+      if (ok) mma_commit_elect(&bars->q_empty);   // q_lat and q_rope (TMEM) may be replaced
     }
+    if (!ok && lane == 0) {
+      give_up();
+      report(p.status, MLA_STATUS_TIMEOUT);
+    }
+    __syncwarp();
+    mma_commit_elect(&bars->qk_done);
+    mbar_drain(&bars->qk_done, 0);   // no MMA may still write TMEM at dealloc
   } else if (warp == 2) {
     // ------------------------------------------------------------ PV issuer
     // O += P . c_KV: M = 128 rows, N = 256 latent columns, K = 64 keys in 4
-    // MMAs, A = P (bf16 pairs) from TMEM, B = the stage's c_KV half (MN-major).
-    if (lane == 0) {
-      const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
-      const uint64_t v_desc0 = sdesc(smem_u32(s_kv), kChunkBytes, 1024, kSwizzle128B);
-      bool ok = true;
-      int g = 0;
-      for (int it = it_begin; ok && it < it_end; ++it) {
-        const int32_t* w = items + (size_t)it * kItemWords;
-        const int n = w[kItPageEnd] - w[kItPageBegin];
-        const int ii = it - it_begin;
-        for (int j = 0; j < n; ++j, ++g) {
-          const int s = g % kStages;
-          if (!mbar_wait(&bars->p_full, g & 1, wc) ||
-              (j == 0 && ii > 0 && !mbar_wait(&bars->o_free, (ii - 1) & 1, wc))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t vd = v_desc0 + (uint64_t)((s * kStageBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16; P (bf16 pairs) from TMEM
-            mma_ts(tmem + kTmemO, tmem + kTmemP + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
-                   (j | kk) != 0);
-          mma_commit(&bars->kv_empty[s]);
-          mma_commit(&bars->o_full);
+    // MMAs, A = P (bf16 pairs) from TMEM buffer g & 1, B = the stage's c_KV
+    // half (MN-major).  Warp-wide loop, one elected lane issues.
+    const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+    const uint64_t v_desc0 = sdesc(smem_u32(s_kv), kChunkBytes, 1024, kSwizzle128B);
+    bool ok = true;
+    int g = 0;
+    for (int it = it_begin; ok && it < it_end; ++it) {
+      const int32_t* w = items + (size_t)it * kItemWords;
+      const int n = w[kItPageEnd] - w[kItPageBegin];
+      const int ii = it - it_begin;
+      for (int j = 0; j < n; ++j, ++g) {
+        const int s = g % kStages;
+        if (!warp_wait(&bars->p_full, g & 1, wc) ||
+            (j == 0 && ii > 0 && !warp_wait(&bars->o_free, (ii - 1) & 1, wc))) {
+          ok = false;
+          break;
         }
-        // o_full alone cannot tell the last page's completion from the one before
-        // (a parity wait sees one phase at a time), so the epilogue waits on this
-        if (ok) mma_commit(&bars->o_done);
+        tc_fence_after();
+        const uint64_t vd = v_desc0 + (uint64_t)((s * kStageBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // 64 keys in steps of 16; P (bf16 pairs) from TMEM
+          mma_ts_elect(tmem + kTmemO, tmem + kTmemP + 32 * (g & 1) + 8 * kk, vd + (uint64_t)(kk * (2048 >> 4)),
+                       idesc_pv, (j | kk) != 0);
+        mma_commit_elect(&bars->kv_empty[s]);
+        mma_commit_elect(&bars->o_full[g & 1]);
       }
-      if (!ok) {
-        give_up();
-        report(p.status, MLA_STATUS_TIMEOUT);
-      }
-      mma_commit(&bars->pv_done);
-      mbar_drain(&bars->pv_done, 0);
+      // o_full alone cannot tell the last page's completion from the one before
+      // (a parity wait sees one phase at a time), so the epilogue waits on this
+      if (ok) mma_commit_elect(&bars->o_done);
     }
+    if (!ok && lane == 0) {
+      give_up();
+      report(p.status, MLA_STATUS_TIMEOUT);
+    }
+    __syncwarp();
+    mma_commit_elect(&bars->pv_done);
+    mbar_drain(&bars->pv_done, 0);
   } else if (warp < kSoftWarp0) {
     // ------------------------------------------------------------ query loader and score sender (4 warps)
     // At each item start the thread of row r copies its 256 q_lat columns and
@@ -411,12 +424,26 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
       const int ii = it - it_begin;
       if (ii > 0 && !warp_wait(&bars->q_empty, (ii - 1) & 1, wc)) goto sender_fail;
       {
+        {
+          const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + ((size_t)w[kItRow] * p.n_heads + r) * 64 +
+                                                             32 * rank);
+          // row r of the K-major A tile, 64 bytes: 16-byte chunk k at (k ^ ((r >> 1) & 3))
+          // (the 64-byte swizzle the MMA descriptor names)
+          uint4 q[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) q[k] = r < p.n_heads ? __ldg(rsrc + k) : make_uint4(0, 0, 0, 0);
+          const uint32_t dst = smem_u32(s_qrope) + r * 64;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) st_shared_v4(dst + ((k ^ ((r >> 1) & 3)) << 4), q[k]);
+          fence_proxy_async_smem();   // read by the tensor cores
+        }
         const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)w[kItRow] * p.n_heads + r) * 512 +
                                                           256 * rank);
 #pragma unroll
@@ -429,17 +456,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           }
           tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        }
-        {
-          const uint4* rsrc = reinterpret_cast<const uint4*>(p.q_rope + ((size_t)w[kItRow] * p.n_heads + r) * 64 +
-                                                             32 * rank);
-          uint32_t v[16];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 q = r < p.n_heads ? __ldg(rsrc + k) : make_uint4(0, 0, 0, 0);
-            v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
-          }
-          tmem_st16(tmem + lane_addr + kTmemQR, v);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -459,7 +475,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (lane == 0) mbar_arrive(&bars->s_read);
         uint32_t hv[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) hv[k] = pack_f16(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+        for (int k = 0; k < 32; ++k)   // scaled to log2 units, then rounded to fp16
+          hv[k] = pack_f16(__uint_as_float(v[2 * k]) * sl2, __uint_as_float(v[2 * k + 1]) * sl2);
         // single tile: page g - 1's own tile must have been read by the softmax and the copy
         if (g >= 1 && !warp_wait(&bars->own_free, (g - 1) & 1, wc)) goto sender_fail;
         {
@@ -496,8 +513,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         const int32_t* w = items + (size_t)it * kItemWords;
         const int n = w[kItPageEnd] - w[kItPageBegin];
         for (int j = 0; j < n; ++j, ++g) {
-          if (!mbar_wait(&bars->own_full, g & 1, wc) ||
-              (g >= 1 && !mbar_wait(&bars->x_sendok, (g - 1) & 1, wc))) {
+          if (!mbar_wait<false, kWaitHintNs>(&bars->own_full, g & 1, wc) ||
+              (g >= 1 && !mbar_wait<false, kWaitHintNs>(&bars->x_sendok, (g - 1) & 1, wc))) {
             ok = false;
             break;
           }
@@ -522,7 +539,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int r = quarter * 32 + lane;
     const int tid = threadIdx.x - kSoftWarp0 * 32;    // 0 .. 255
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const float sl2 = p.scale_log2;
     const uint32_t x_sendok_peer = mapa(smem_u32(&bars->x_sendok), peer);
     bool out_of_range = false;   // a fp16 partial overflowed: a reference max of +Inf, or a NaN sum
     // The sequence length of the next item is loaded one item ahead, so that
@@ -574,37 +590,40 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             mbar_arrive_relaxed_cluster(ok_addr);
           }
         }
-        float sc[32];
+        // scores in log2 units: fp16(own) + fp16(peer), summed as fp16 pairs
+        uint32_t s2[16];
         {
           const uint32_t* ow = reinterpret_cast<const uint32_t*>(po);
           const uint32_t* pw = reinterpret_cast<const uint32_t*>(pr);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) add_f16x2_to_f32(ow[k], pw[k], sc[2 * k], sc[2 * k + 1]);
+          for (int k = 0; k < 16; ++k) s2[k] = hadd2(ow[k], pw[k]);
         }
-        // masked columns [0, lo) of this page: the last page's zero fill, or all
-        // of them when the device seq_lens disagree with the plan
+        // masked keys [0, lo) of this page (-inf): the last page's zero fill, or
+        // all of them when the device seq_lens disagree with the plan
         const int lo = stale ? kPage : (j == n - 1 ? shift_last : 0);
         if (lo > 32 * c) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (32 * c + k < lo) sc[k] = -CUDART_INF_F;
+          for (int k = 0; k < 16; ++k) {
+            if (32 * c + 2 * k < lo) s2[k] = (s2[k] & 0xffff0000u) | 0xfc00u;
+            if (32 * c + 2 * k + 1 < lo) s2[k] = (s2[k] & 0x0000ffffu) | 0xfc000000u;
+          }
         }
         float mloc;
         {
-          float t[11], u[4];
+          uint32_t t[8];
 #pragma unroll
-          for (int k = 0; k < 10; ++k) t[k] = fmax3(sc[3 * k], sc[3 * k + 1], sc[3 * k + 2]);
-          t[10] = fmaxf(sc[30], sc[31]);
+          for (int k = 0; k < 8; ++k) t[k] = hmax2(s2[k], s2[k + 8]);
 #pragma unroll
-          for (int k = 0; k < 3; ++k) u[k] = fmax3(t[3 * k], t[3 * k + 1], t[3 * k + 2]);
-          u[3] = fmaxf(t[9], t[10]);
-          mloc = fmaxf(fmax3(u[0], u[1], u[2]), u[3]);
+          for (int k = 0; k < 4; ++k) t[k] = hmax2(t[k], t[k + 4]);
+          t[0] = hmax2(hmax2(t[0], t[2]), hmax2(t[1], t[3]));
+          const float2 m2 = unpack_f16x2(t[0]);
+          mloc = fmaxf(m2.x, m2.y);
         }
         s_pmax[(b * 2 + c) * kRows + r] = mloc;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->pmax[b][quarter]);
         if (!warp_wait(&bars->pmax[b][quarter], (gj >> 1) & 1, wc)) goto softmax_fail;
-        const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kRows + r]) * sl2;
+        const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kRows + r]);
 
         // lazy reference max (log2 domain): move it only when the row max grows by > 2^8
         const float m_new = fmaxf(m_ref, mx);
@@ -620,16 +639,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float e0 = ex2(fmaf(sc[2 * k], sl2, nb));
-          const float e1 = ex2(fmaf(sc[2 * k + 1], sl2, nb));
+          float x0, x1;
+          add_f16x2_to_f32(s2[k], nb, x0, x1);   // exact score + nb, rounded once
+          const float e0 = ex2(x0), e1 = ex2(x1);
           pk[k] = pack_bf16(e0, e1);
           ps[k & 3] += e0 + e1;
         }
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
 
-        // the single P buffer is free once the previous page's PV product has completed
-        if (gj >= 1 && !warp_wait(&bars->o_full, (gj - 1) & 1, wc)) goto softmax_fail;
+        // P buffer gj & 1 is free once the PV product of page gj - 2 has completed
+        if (gj >= 2 && !warp_wait(&bars->o_full[gj & 1], ((gj >> 1) - 1) & 1, wc)) goto softmax_fail;
         if (__any_sync(0xffffffffu, move && j > 0)) {
+          // rescaling O: the PV product of page gj - 1 (same item) must have landed
+          if (!warp_wait(&bars->o_full[(gj - 1) & 1], ((gj - 1) >> 1) & 1, wc)) goto softmax_fail;
           tc_fence_after();
           const float a = (move && j > 0) ? alpha : 1.f;
 #pragma unroll 1
@@ -643,7 +665,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           }
           tmem_st_wait();
         }
-        tmem_st16(tmem + lane_addr + kTmemP + 16 * c, pk);   // keys [32c, 32c+32) as bf16 pairs
+        tmem_st16(tmem + lane_addr + kTmemP + 32 * (gj & 1) + 16 * c, pk);   // keys [32c, 32c+32), bf16 pairs
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -652,7 +674,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 
       // epilogue: O / l  ->  o_lat (whole row) or the row's partial slot.  A
       // stale item has P = 0 throughout: its row is written as zeros.
-      out_of_range |= (m_ref == CUDART_INF_F) | (l_run != l_run);
       {
         if (!warp_wait(&bars->o_done, ii & 1, wc)) goto softmax_fail;
         tc_fence_after();
@@ -662,7 +683,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         if (lane == 0) mbar_arrive(&bars->lsum[quarter]);
         if (!warp_wait(&bars->lsum[quarter], ii & 1, wc)) goto softmax_fail;
         l_run = ls[r] + ls[kRows + r];             // same order in both halves
-        out_of_range |= (l_run != l_run);
+        out_of_range |= (m_ref == CUDART_INF_F) | (l_run != l_run);
         const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
         const bool valid = r < p.n_heads;
         const bool o_lat_32b = (reinterpret_cast<uintptr_t>(p.o_lat) & 31) == 0;

@@ -106,18 +106,53 @@ struct WaitCtl {
   unsigned long long limit_ns; // bound of each wait
 };
 
-// mbar_wait with the abort flag and the limit read from `ctl` on the slow path.
-template <bool kClusterAcquire = false>
+// try_wait that may suspend the thread for up to `hint_ns` (it resumes as soon
+// as the phase completes), so that a waiting warp takes no issue slots.
+template <bool kClusterAcquire>
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  if (kClusterAcquire)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with the abort flag and the limit read from `ctl` after every
+// unsuccessful (suspending) poll.
+template <bool kClusterAcquire = false, uint32_t kHintNs = 0>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile WaitCtl* ctl) {
-  if (kClusterAcquire ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity))
-    return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
+  if (kHintNs == 0) {
     if (kClusterAcquire ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity))
       return true;
-    if ((i & 15) == 0) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+      if (kClusterAcquire ? mbar_try_wait_acq_cluster(bar, parity) : mbar_try_wait(bar, parity))
+        return true;
+      if ((i & 15) == 0) {
+        if (ctl->abort) return false;
+        if (globaltimer() - t0 > ctl->limit_ns) return false;
+      }
+    }
+  } else {
+    if (mbar_try_wait_hint<kClusterAcquire>(bar, parity, kHintNs)) return true;
+    const uint64_t t0 = globaltimer();
+    for (;;) {
       if (ctl->abort) return false;
       if (globaltimer() - t0 > ctl->limit_ns) return false;
+      if (mbar_try_wait_hint<kClusterAcquire>(bar, parity, kHintNs)) return true;
     }
   }
 }
@@ -174,6 +209,12 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
 }
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// 16-byte shared-memory store at a shared::cta address.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // 32-byte global store of eight words (address 32-byte aligned).
@@ -314,11 +355,47 @@ __device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// The same, issued by one elected lane of a converged warp: the whole warp
+// computes the (warp-uniform) operands and a single thread issues.
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T from one elected lane of a converged warp.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when all previously issued tcgen05 async ops of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// mma_commit from one elected lane of a converged warp (the lane that issued
+// the warp's MMAs: elect.sync picks the same lane while the warp is converged).
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld_wait() {
@@ -354,6 +431,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+// One 32-bit column: thread i of the warp reads / writes lane (base_lane + i).
+// The load waits for its own completion.
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\ttcgen05.wait::ld.sync.aligned;"
+               : "=r"(r)
+               : "r"(taddr)
+               : "memory");
+  return r;
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
