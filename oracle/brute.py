@@ -13,11 +13,13 @@ from __future__ import annotations
 import math
 
 
-def brute_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q, scale):
+def brute_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q, scale, visible=None):
     """Nested lists in, nested lists out.
 
     q_nope[n][h][d], q_rope[n][h][r], caches[b][t][k + r] (latent then rope),
     W_UK[k][h][d], W_UV[k][h][v].  Returns (out[n][h][v], lse[n][h]).
+    ``visible`` (optional): visible[b][i] is the list of key positions query
+    i of sequence b attends, in place of 0 .. T - s + i.
     """
     n_rows = len(q_nope)
     H = len(q_nope[0])
@@ -31,10 +33,10 @@ def brute_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q, scale):
         T = len(cache)
         for i in range(s_q):
             n = b * s_q + i
-            last = T - s_q + i
+            keys = list(range(T - s_q + i + 1)) if visible is None else list(visible[b][i])
             for h in range(H):
                 logits = []
-                for t in range(last + 1):
+                for t in keys:
                     acc = 0.0
                     for j in range(d):
                         kj = 0.0
@@ -50,10 +52,10 @@ def brute_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q, scale):
                 lse[n][h] = m + math.log(z)
                 for j in range(v):
                     acc = 0.0
-                    for t in range(last + 1):
+                    for a, t in enumerate(keys):
                         vj = 0.0
                         for c in range(dc):
                             vj += cache[t][c] * W_UV[c][h][j]
-                        acc += (w[t] / z) * vj
+                        acc += (w[a] / z) * vj
                     out[n][h][j] = acc
     return out, lse

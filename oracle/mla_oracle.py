@@ -206,6 +206,30 @@ def masked_softmax(logits: np.ndarray, keep: np.ndarray):
     return e / z, (m + np.log(z))[..., 0]
 
 
+def tree_masks(parents) -> list[int]:
+    """Visibility bitmasks of a speculative token tree (EAGLE-style drafts).
+
+    The Perplexity write-up ("Будущая работа" / future work) names EAGLE-style
+    speculative decoding that drafts several tokens as a tree.  The pages do
+    not write the attention mask out; the plain reading, used here: draft
+    token i sees the committed prefix, every ancestor of i in the tree, and
+    itself.  ``parents[i]`` is the index of token i's parent among the drafts
+    (< i), or -1 when its parent is the last committed token.  Bit j of the
+    result's entry i is set iff draft j is visible to draft i.  A chain
+    (parents = [-1, 0, 1, ...]) gives the causal masks, a star (all -1) lets
+    every draft see only itself.
+    """
+    masks = []
+    for i, par in enumerate(parents):
+        if not -1 <= par < i:
+            raise ValueError(f"parent of draft {i} must be in [-1, {i})")
+        m = 1 << i
+        if par >= 0:
+            m |= masks[par]
+        masks.append(m)
+    return masks
+
+
 def default_scale(d_nope: int = D_NOPE, d_rope: int = D_ROPE) -> float:
     """1/sqrt(d_nope + d_rope): the plain reading for the unstated scale."""
     return 1.0 / math.sqrt(d_nope + d_rope)
@@ -216,7 +240,7 @@ def default_scale(d_nope: int = D_NOPE, d_rope: int = D_ROPE) -> float:
 # --------------------------------------------------------------------------
 def mla_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q: int, scale: float | None = None,
                heads=None, chunk: int = 2048, counter: FlopCounter | None = None,
-               with_intermediates: bool = True):
+               with_intermediates: bool = True, draft_masks=None):
     """Un-absorbed (order 1) MLA decode attention over per-sequence caches.
 
     Arguments (all converted to float64):
@@ -231,6 +255,11 @@ def mla_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q: int, scale: float | None
       logit[t] = scale * (q_nope . K_t + q_rope . k_rope_t) (RoPE-MQA score added)
       keep t <= T_b - s_q + i;  p = softmax(logit)         (standard softmax)
       out = sum_t p[t] V_t                                  (§3.1 Step 2)
+
+    ``draft_masks`` (optional, one list of s_q bitmasks per sequence, e.g.
+    from :func:`tree_masks`) replaces the causal rule among the s_q new
+    tokens: query i keeps every prefix key t < T_b - s_q and new token j
+    (key T_b - s_q + j) iff bit j of draft_masks[b][i] is set.
 
     Returns a dict with 'out' (N,h',v), 'lse' (N,h') natural-log LSE of the
     scaled logits, and (if ``with_intermediates``) the order-2 intermediates
@@ -280,7 +309,13 @@ def mla_decode(q_nope, q_rope, caches, W_UK, W_UV, s_q: int, scale: float | None
         logits *= scale
 
         pos = np.arange(T)
-        keep = pos[None, :] <= (T - s_q + np.arange(s_q))[:, None]      # (s, T)
+        if draft_masks is None:
+            keep = pos[None, :] <= (T - s_q + np.arange(s_q))[:, None]  # (s, T): causal
+        else:
+            keep = np.ones((s_q, T), dtype=bool)                         # prefix: all visible
+            for i in range(s_q):
+                for j in range(s_q):
+                    keep[i, T - s_q + j] = bool((int(draft_masks[b][i]) >> j) & 1)
         p, l = masked_softmax(logits, keep[None, :, :])                  # (h, s, T)
 
         acc = np.zeros((1, H, s_q, v))
