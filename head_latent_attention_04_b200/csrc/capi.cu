@@ -244,7 +244,33 @@ mla_status_t mla_decode_attn(const mla_dims_t* dims, const void* q_lat, const vo
   // checks slots against the plan, the host cannot see the device plan here.
   if ((o_part && !aligned16(o_part)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
     return set_error(MLA_ERR_INVALID_ARG, "o_part must be 16-byte aligned, lse_part 4-byte aligned");
-  return launch_decode_attn(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens,
+  return launch_decode_attn(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens, nullptr,
+                            static_cast<const int32_t*>(plan_dev), num_clusters, o_part, lse_part,
+                            o_lat, lse_out, status, stream);
+}
+
+mla_status_t mla_decode_attn_tree(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                                  const void* kv_pool, const int32_t* block_table, const int32_t* seq_lens,
+                                  const int32_t* draft_masks, const void* plan_dev, int32_t num_clusters,
+                                  float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                                  int32_t* status, void* stream) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  if (dims->causal != 0)
+    return set_error(MLA_ERR_INVALID_ARG, "draft-tree attention needs dims->causal = 0 (plan with kv_len = T)");
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  MLA_TRY(check_ptr(q_rope, "q_rope"));
+  MLA_TRY(check_ptr(kv_pool, "kv_pool"));
+  MLA_TRY(check_ptr(block_table, "block_table"));
+  MLA_TRY(check_ptr(seq_lens, "seq_lens"));
+  MLA_TRY(check_ptr(draft_masks, "draft_masks"));
+  MLA_TRY(check_ptr(plan_dev, "plan_dev"));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  if (num_clusters < 1 || num_clusters > 4096)
+    return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
+  if ((o_part && !aligned16(o_part)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
+    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 16-byte aligned, lse_part 4-byte aligned");
+  return launch_decode_attn(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_masks,
                             static_cast<const int32_t*>(plan_dev), num_clusters, o_part, lse_part,
                             o_lat, lse_out, status, stream);
 }

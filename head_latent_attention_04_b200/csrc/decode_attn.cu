@@ -88,6 +88,7 @@ struct DecodeParams {
   const int32_t* block_table;   // [B][max_blocks]
   const int32_t* seq_lens;      // [B]
   const int32_t* plan;
+  const int32_t* draft_masks;   // [B][s_q] visibility of the drafts (bit j: draft j), or null
   float* o_part;                // [slots][H][512]
   float* lse_part;              // [slots][H]
   __nv_bfloat16* o_lat;         // [N][H][512]
@@ -543,15 +544,29 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     bool out_of_range = false;   // a fp16 partial overflowed: a reference max of +Inf, or a NaN sum
     // The sequence length of the next item is loaded one item ahead, so that
     // the stale-plan check never waits for memory at an item boundary.
-    int T_next = it_begin < it_end ? p.seq_lens[items[(size_t)it_begin * kItemWords + kItB]] : 0;
+    // So is the next item's draft mask, when drafts form a tree.
+    const bool tree = p.draft_masks != nullptr;
+    int T_next = 0, m_next = 0;
+    if (it_begin < it_end) {
+      const int32_t* w0 = items + (size_t)it_begin * kItemWords;
+      T_next = p.seq_lens[w0[kItB]];
+      if (tree) m_next = p.draft_masks[w0[kItRow]];
+    }
     int g = 0;
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
-      const int row = w[kItRow], slot = w[kItSlot];
-      const int n = w[kItPageEnd] - w[kItPageBegin];
+      const int row = w[kItRow], slot = w[kItSlot], pb = w[kItPageBegin];
+      const int n = w[kItPageEnd] - pb;
       const int ii = it - it_begin;
       const bool stale = item_stale(w, T_next, p);
-      if (it + 1 < it_end) T_next = p.seq_lens[items[(size_t)(it + 1) * kItemWords + kItB]];
+      const uint32_t drafts_seen = (uint32_t)m_next;
+      if (it + 1 < it_end) {
+        const int32_t* w1 = items + (size_t)(it + 1) * kItemWords;
+        T_next = p.seq_lens[w1[kItB]];
+        if (tree) m_next = p.draft_masks[w1[kItRow]];
+      }
+      // key index of the first draft (the plan of a tree batch is not causal: kv_len = T)
+      const int first_draft = w[kItKvLen] - p.s_q;
       if (stale && tid == 0 && rank == 0) report(p.status, MLA_STATUS_BAD_SEQLEN);
       // keys masked in the item's last page: the zero-filled rows of its shifted load
       const int shift_last = kPage - min(last_page_keys(w), kPage);
@@ -606,6 +621,19 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           for (int k = 0; k < 16; ++k) {
             if (32 * c + 2 * k < lo) s2[k] = (s2[k] & 0xffff0000u) | 0xfc00u;
             if (32 * c + 2 * k + 1 < lo) s2[k] = (s2[k] & 0x0000ffffu) | 0xfc000000u;
+          }
+        }
+        if (tree) {
+          // draft keys: column col holds key (page start + col - shift); draft
+          // d = key - first_draft is visible iff bit d of this row's mask is set
+          const int col0 = first_draft - ((pb + j) * kPage - (j == n - 1 ? shift_last : 0));
+          if (col0 < 32 * c + 32) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const int d0 = 32 * c + 2 * k - col0, d1 = d0 + 1;
+              if (d0 >= 0 && !((drafts_seen >> d0) & 1u)) s2[k] = (s2[k] & 0xffff0000u) | 0xfc00u;
+              if (d1 >= 0 && !((drafts_seen >> d1) & 1u)) s2[k] = (s2[k] & 0x0000ffffu) | 0xfc000000u;
+            }
           }
         }
         float mloc;
@@ -776,7 +804,7 @@ cudaError_t decode_smem_attr() {
 
 mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
                                 const void* kv_pool, const int32_t* block_table,
-                                const int32_t* seq_lens, const int32_t* plan_dev,
+                                const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream) {
   // The pool as (column, row within the block, block): a box may start at a
@@ -798,6 +826,7 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
   p.block_table = block_table;
   p.seq_lens = seq_lens;
   p.plan = plan_dev;
+  p.draft_masks = draft_masks;
   p.o_part = o_part;
   p.lse_part = lse_part;
   p.o_lat = static_cast<__nv_bfloat16*>(o_lat);

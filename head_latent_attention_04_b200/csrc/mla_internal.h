@@ -51,7 +51,7 @@ mla_status_t launch_out_uv_fp8(const void* o_lat, const void* w_codes, const flo
                                int n_tokens, int n_heads, void* stream);
 mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
                                 const void* kv_pool, const int32_t* block_table,
-                                const int32_t* seq_lens, const int32_t* plan_dev,
+                                const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream);
 mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,

@@ -113,7 +113,7 @@ mla_status_t decode_attn_combine_noalloc(const mla_dims_t& d, const void* q_lat,
 
   cudaError_t e = cudaMemcpyAsync(plan_dev, plan_host, words * 4, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "plan copy: %s", cudaGetErrorString(e));
-  st = launch_decode_attn(d, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_dev, num_clusters, o_part,
+  st = launch_decode_attn(d, q_lat, q_rope, kv_pool, block_table, seq_lens, nullptr, plan_dev, num_clusters, o_part,
                           lse_part, o_lat, lse_out, status, stream);
   if (st != MLA_OK) return st;
   if (slots > 0)

@@ -28,7 +28,7 @@ EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
            "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes",
            "mla_quantize_w_uk_fp8", "mla_quantize_w_uv_fp8", "mla_quantize_rows_fp8", "mla_absorb_q_fp8",
-           "mla_out_uv_fp8", "mla_set_wait_limit_ns")
+           "mla_out_uv_fp8", "mla_set_wait_limit_ns", "mla_decode_attn_tree")
 
 
 class MlaDims(ctypes.Structure):
@@ -50,6 +50,7 @@ for _name, _args in {
     "mla_plan_size": [_pdims, _i32, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
     "mla_plan": [_pdims, _vp, _i32, _vp, _sz, ctypes.POINTER(_i32)],
     "mla_decode_attn": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
+    "mla_decode_attn_tree": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_combine": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_debug_gather_pages": [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "mla_decode_attn_combine_noalloc": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _vp, _vp, _vp, _vp],
@@ -224,6 +225,16 @@ def decode_attn(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, plan_dev, n
                                 _ptr(status), _stream(stream)), "mla_decode_attn")
 
 
+def decode_attn_tree(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_masks, plan_dev, num_clusters,
+                     o_part, lse_part, o_lat, lse_out=None, status=None, stream=None):
+    """decode_attn for drafts that form a tree: ``draft_masks`` int32 [B][s_q]
+    (device), bit j of row i = draft j visible to query i (dims.causal must be 0)."""
+    _check(_lib.mla_decode_attn_tree(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(kv_pool),
+                                     _ptr(block_table), _ptr(seq_lens), _ptr(draft_masks), _ptr(plan_dev),
+                                     num_clusters, _ptr(o_part), _ptr(lse_part), _ptr(o_lat), _ptr(lse_out),
+                                     _ptr(status), _stream(stream)), "mla_decode_attn_tree")
+
+
 def combine(dims, plan_dev, o_part, lse_part, o_lat, lse_out=None, stream=None):
     _check(_lib.mla_combine(ctypes.byref(dims), _ptr(plan_dev), _ptr(o_part), _ptr(lse_part),
                             _ptr(o_lat), _ptr(lse_out), _stream(stream)), "mla_combine")
@@ -303,14 +314,22 @@ class Decoder:
         self.fp8_uk = quantize_w_uk_fp8(w_uk, stream)
         self.fp8_uv = quantize_w_uv_fp8(w_uv, stream)
 
-    def run(self, q_nope, q_rope, kv_pool, block_table, w_uk, w_uv, stream=None) -> DecodeOutputs:
+    def run(self, q_nope, q_rope, kv_pool, block_table, w_uk, w_uv, stream=None,
+            draft_masks=None) -> DecodeOutputs:
+        """``draft_masks`` (device int32 [B][s_q], only with causal=False): the
+        drafts form a tree, see :func:`decode_attn_tree`."""
         if self.fp8_uk is not None:
             absorb_q_fp8(q_nope, self.fp8_uk, self.q_lat, stream)
         else:
             absorb_q(q_nope, w_uk, self.q_lat, stream)
-        decode_attn(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev,
-                    self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
-                    self.lse, self.status, stream)
+        if draft_masks is not None:
+            decode_attn_tree(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev, draft_masks,
+                             self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
+                             self.lse, self.status, stream)
+        else:
+            decode_attn(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev,
+                        self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
+                        self.lse, self.status, stream)
         if self.num_slots > 0:
             combine(self.dims, self.plan_dev, self.o_part, self.lse_part, self.o_lat, self.lse, stream)
         if self.fp8_uv is not None:

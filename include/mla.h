@@ -209,6 +209,29 @@ mla_status_t mla_decode_attn(const mla_dims_t* dims, const void* q_lat, const vo
                              int32_t* status, void* stream);
 
 /*
+ * mla_decode_attn_tree -- mla_decode_attn for drafted tokens that form a tree
+ * (EAGLE-style speculative decoding, named as future work in "Lower latency
+ * and higher throughput with multi-node DeepSeek deployment", section
+ * "Будущая работа": several tokens drafted as a tree instead of a chain).
+ * Query i of sequence b attends every committed key t < T_b - s_q and the
+ * drafts its mask allows:
+ *   draft_masks  int32 [B][s_q] (device): bit j of draft_masks[b * s_q + i]
+ *                set = key T_b - s_q + j (draft j) is visible to query i.
+ *                For a tree, row i holds i's ancestors and i itself; the
+ *                causal rule is the chain's masks (bits 0 .. i).
+ * The plan must be made with dims->causal = 0 (every row covers all T_b
+ * keys; MLA_ERR_INVALID_ARG otherwise).  A row whose mask and prefix leave
+ * no key visible is written as zeros with LSE -inf.  1 <= s_q <= 8.  All
+ * other arguments and outputs are those of mla_decode_attn; mla_combine
+ * completes split rows as usual.
+ */
+mla_status_t mla_decode_attn_tree(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                                  const void* kv_pool, const int32_t* block_table, const int32_t* seq_lens,
+                                  const int32_t* draft_masks, const void* plan_dev, int32_t num_clusters,
+                                  float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                                  int32_t* status, void* stream);
+
+/*
  * mla_combine -- log-sum-exp merge of the split pieces of each split row:
  *   L = log sum_i exp(lse_i),  o_lat = sum_i exp(lse_i - L) * O_i.
  * Reads o_part/lse_part written by mla_decode_attn with the same plan, writes

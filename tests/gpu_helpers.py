@@ -30,13 +30,14 @@ def run_gpu(w: W.Workload, num_clusters=None, causal=True):
     return dec, res
 
 
-def oracle_rows(w: W.Workload, b: int, heads=None):
-    """Oracle for sequence b (all its s_q rows), optionally a head subset."""
+def oracle_rows(w: W.Workload, b: int, heads=None, draft_masks=None):
+    """Oracle for sequence b (all its s_q rows), optionally a head subset and
+    the drafts' visibility masks (one list of s_q bitmasks)."""
     rows = slice(b * w.s_q, (b + 1) * w.s_q)
     cache = w.cache_rows(b).cpu().double().numpy()
     return O.mla_decode(w.q_nope[rows].cpu().double().numpy(), w.q_rope[rows].cpu().double().numpy(),
                         [cache], w.w_uk.cpu().double().numpy(), w.w_uv.cpu().double().numpy(),
-                        w.s_q, heads=heads)
+                        w.s_q, heads=heads, draft_masks=None if draft_masks is None else [draft_masks])
 
 
 def oracle_all(w: W.Workload):

@@ -212,6 +212,17 @@ def test_noalloc_refuses_plans_that_do_not_match():
     assert _noalloc(dims, other_h, other_h.nbytes, 8) == mla.MLA_ERR_INVALID_ARG
 
 
+def test_tree_entry_point_needs_a_non_causal_plan():
+    causal = mla.make_dims(2, 4, 16, 4, 8, causal=True)
+    r = mla._lib.mla_decode_attn_tree(ctypes.byref(causal), 16, 16, 16, 16, 16, 16, 16, 4, None, None, 16,
+                                      None, None, None)
+    assert r == mla.MLA_ERR_INVALID_ARG and b"causal" in mla._lib.mla_last_error_string()
+    flat = mla.make_dims(2, 4, 16, 4, 8, causal=False)
+    r = mla._lib.mla_decode_attn_tree(ctypes.byref(flat), 16, 16, 16, 16, 16, None, 16, 4, None, None, 16,
+                                      None, None, None)
+    assert r == mla.MLA_ERR_INVALID_ARG and b"draft_masks" in mla._lib.mla_last_error_string()
+
+
 def test_fp8_entry_points_validate_before_any_launch():
     lib = mla._lib
     assert lib.mla_quantize_w_uk_fp8(16, 0, 16, 16, None) == mla.MLA_ERR_UNSUPPORTED        # n_heads
