@@ -242,8 +242,8 @@ mla_status_t mla_decode_attn(const mla_dims_t* dims, const void* q_lat, const vo
     return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
   // o_part / lse_part may be NULL only when the plan splits no row; the kernel
   // checks slots against the plan, the host cannot see the device plan here.
-  if ((o_part && !aligned16(o_part)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
-    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 16-byte aligned, lse_part 4-byte aligned");
+  if ((o_part && (reinterpret_cast<uintptr_t>(o_part) & 31u)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
+    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 32-byte aligned, lse_part 4-byte aligned");
   return launch_decode_attn(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens, nullptr,
                             static_cast<const int32_t*>(plan_dev), num_clusters, o_part, lse_part,
                             o_lat, lse_out, status, stream);
@@ -268,8 +268,8 @@ mla_status_t mla_decode_attn_tree(const mla_dims_t* dims, const void* q_lat, con
   MLA_TRY(check_ptr(o_lat, "o_lat"));
   if (num_clusters < 1 || num_clusters > 4096)
     return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
-  if ((o_part && !aligned16(o_part)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
-    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 16-byte aligned, lse_part 4-byte aligned");
+  if ((o_part && (reinterpret_cast<uintptr_t>(o_part) & 31u)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
+    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 32-byte aligned, lse_part 4-byte aligned");
   return launch_decode_attn(*dims, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_masks,
                             static_cast<const int32_t*>(plan_dev), num_clusters, o_part, lse_part,
                             o_lat, lse_out, status, stream);

@@ -737,12 +737,17 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
                 reinterpret_cast<uint4*>(dst)[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
             }
           } else {
-            // column-group-major partials: a warp's 32 rows of one 4-column group are contiguous
-            float4* dst = reinterpret_cast<float4*>(p.o_part) + ((size_t)slot * 128 + col / 4) * p.n_heads + r;
+            // column-group-major partials, 8 columns (32 bytes) per group: a warp's
+            // 32 rows of one group are 1 KB contiguous, and a reader of one row
+            // gets whole 32-byte sectors
+            float* dst = p.o_part + (((size_t)slot * 64 + col / 8) * p.n_heads + r) * 8;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              dst[(size_t)k * p.n_heads] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
-                                   __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+            for (int k = 0; k < 4; ++k) {
+              uint32_t v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = __float_as_uint(__uint_as_float(o[8 * k + e]) * inv_l);
+              st_global_v8(dst + (size_t)k * p.n_heads * 8, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+            }
           }
         }
         if (valid && rank == 0 && c == 0) {

@@ -187,9 +187,11 @@ mla_status_t mla_plan(const mla_dims_t* dims, const int32_t* seq_lens_host, int3
  *                plan (mla_plan, host only, microseconds) and copies it each step.
  *   plan_dev     the plan from mla_plan, copied to the device
  *   num_clusters the num_clusters the plan was built for (grid = 2 * num_clusters CTAs)
- *   o_part       fp32, slots x n_heads x 512  workspace (split rows); element
- *                (slot, h, col) at ((slot*128 + col/4)*n_heads + h)*4 + col%4,
- *                so that the stores of 32 rows are contiguous
+ *   o_part       fp32, slots x n_heads x 512  workspace (split rows), 32-byte
+ *                aligned; element (slot, h, col) at
+ *                ((slot*64 + col/8)*n_heads + h)*8 + col%8, so that the stores
+ *                of 32 rows are contiguous and a reader of one row gets whole
+ *                32-byte sectors
  *   lse_part     fp32 [slots][n_heads]        workspace
  *   o_lat        bf16 [N][n_heads][512]       rows not split are written here
  *   lse_out      fp32 [N][n_heads] or NULL    natural-log LSE of the scaled logits
