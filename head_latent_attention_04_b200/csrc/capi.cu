@@ -309,6 +309,47 @@ mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void*
 
 size_t mla_noalloc_scratch_bytes(void) { return noalloc_scratch_bytes(); }
 
+static mla_status_t check_prefill(int T, int s, int n_heads, int num_blocks) {
+  if (n_heads < 1 || n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
+  if (T < 1 || T > (1 << 22)) return set_error(MLA_ERR_UNSUPPORTED, "T must be in [1, 2^22]");
+  if (s < 1 || s > T) return set_error(MLA_ERR_INVALID_ARG, "s must be in [1, T]");
+  if (num_blocks < 1 || (int64_t)num_blocks * 64 > INT32_MAX)
+    return set_error(MLA_ERR_INVALID_ARG, "num_blocks out of range");
+  return MLA_OK;
+}
+
+mla_status_t mla_prefill_up_proj(const void* kv_pool, const int32_t* block_table_row, int32_t T, int32_t num_blocks,
+                                 const void* w_uk, const void* w_uv, int32_t n_heads, void* k_out, void* v_out,
+                                 void* stream) {
+  clear_error();
+  MLA_TRY(check_prefill(T, 1, n_heads, num_blocks));
+  MLA_TRY(check_ptr(kv_pool, "kv_pool"));
+  MLA_TRY(check_ptr(block_table_row, "block_table_row"));
+  MLA_TRY(check_ptr(w_uk, "w_uk"));
+  MLA_TRY(check_ptr(w_uv, "w_uv"));
+  MLA_TRY(check_ptr(k_out, "k_out"));
+  MLA_TRY(check_ptr(v_out, "v_out"));
+  return launch_prefill_up_proj(kv_pool, block_table_row, T, num_blocks, w_uk, w_uv, n_heads, k_out, v_out, stream);
+}
+
+mla_status_t mla_prefill_attn(const void* q_nope, const void* q_rope, const void* k, const void* v,
+                              const void* kv_pool, const int32_t* block_table_row, int32_t T, int32_t s,
+                              int32_t n_heads, int32_t num_blocks, float scale, void* out, float* lse, void* stream) {
+  clear_error();
+  MLA_TRY(check_prefill(T, s, n_heads, num_blocks));
+  if (!(scale > 0.f) || scale != scale) return set_error(MLA_ERR_INVALID_ARG, "scale must be > 0");
+  MLA_TRY(check_ptr(q_nope, "q_nope"));
+  MLA_TRY(check_ptr(q_rope, "q_rope"));
+  MLA_TRY(check_ptr(k, "k"));
+  MLA_TRY(check_ptr(v, "v"));
+  MLA_TRY(check_ptr(kv_pool, "kv_pool"));
+  MLA_TRY(check_ptr(block_table_row, "block_table_row"));
+  MLA_TRY(check_ptr(out, "out"));
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return set_error(MLA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  return launch_prefill_attn(q_nope, q_rope, k, v, kv_pool, block_table_row, T, s, n_heads, num_blocks, scale, out,
+                             lse, stream);
+}
+
 void mla_set_wait_limit_ns(int64_t ns) { set_decode_wait_limit_ns(ns); }
 
 mla_status_t mla_debug_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,

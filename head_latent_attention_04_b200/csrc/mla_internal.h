@@ -57,6 +57,12 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
 mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,
                             const float* o_part, const float* lse_part, void* o_lat,
                             float* lse_out, void* stream);
+mla_status_t launch_prefill_up_proj(const void* kv_pool, const int32_t* block_row, int T, int num_blocks,
+                                    const void* w_uk, const void* w_uv, int n_heads, void* k_out, void* v_out,
+                                    void* stream);
+mla_status_t launch_prefill_attn(const void* q_nope, const void* q_rope, const void* k, const void* v,
+                                 const void* kv_pool, const int32_t* block_row, int T, int s, int n_heads,
+                                 int num_blocks, float scale, void* out, float* lse, void* stream);
 mla_status_t launch_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
                                  int32_t n_pages, int32_t max_blocks, int32_t num_blocks, void* out,
                                  int32_t* status, void* stream);

@@ -1,0 +1,517 @@
+// Prefill / chunked prefill of MLA in order 1 ("MHA form") on sm_100a.
+//
+// "MLA Matrix Absorption Analysis" section 2.4.1 compares the evaluation
+// orders of the first absorption: when the query length equals the key
+// length (t = s, prefill) order 1 needs fewer FLOPs than the absorbed order
+// (by 98304 s^2 at DeepSeek-V3 widths); the Perplexity write-up's future-work
+// section names prefill in the up-projected form and chunked prefill.  So
+// prefill up-projects the latent cache once per sequence,
+//   K[t,h,:] = W_UK[:,h,:]^T c_KV[t]     (notes section 2.1 Step 2)
+//   V[t,h,:] = W_UV[:,h,:]^T c_KV[t]     (notes section 3.1 Step 1)
+// and runs causal multi-head attention with the RoPE key shared by all heads:
+//   logit[i,h,t] = scale (q_nope[i,h] . K[t,h] + q_rope[i,h] . k_rope[t])
+//   out[i,h,:]   = sum_t softmax_t(logit) V[t,h,:]     over t <= T - s + i
+// (the s new tokens of a chunk are already in the cache and sit at positions
+// T - s .. T - 1, so a chunk of s < T tokens is chunked prefill).
+//
+// up_proj_kernel: one CTA per (K or V, head, 128-token tile): a swap-AB
+//   tcgen05 GEMM, M = 128 features of the head's W_UK / W_UV slice, N = 128
+//   tokens (two cache pages, read through the block table by TMA from the
+//   (column, row, block) view of the pool), K = 512 latent columns streamed
+//   through a ring; the TMA-store epilogue writes K or V [T][h][128] bf16.
+// prefill_attn_kernel: one CTA per (128-query tile, head).  Warp 0 stages
+//   the Q tile once and K / k_rope / V tiles of 128 keys through a two-stage
+//   ring; warp 1 issues S = Q K^T (M = 128 queries, N = 128 keys, K = 192:
+//   8 MMAs on K, 4 on k_rope) into a single S buffer; warp 2 issues
+//   O += P V (M = 128, N = 128, K = 128 keys: 8 MMAs) from two P buffers;
+//   warps 3-6 run the online softmax, one thread per query row (TMEM lane
+//   quarter = warp % 4), with the causal mask on the diagonal tiles and a
+//   lazy reference maximum, and write the normalised rows.
+// TMEM (512 columns): S [0,128) fp32, P [128,192) and [192,256) bf16 pairs,
+// O [256,384) fp32.
+#include "mla_internal.h"
+#include "ptx.cuh"
+#include "tmap.h"
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+namespace mla {
+namespace {
+
+using namespace ptx;
+
+constexpr int kTile = 128;                 // tokens per tile (queries, keys, up-projection)
+constexpr int kChunk = kTile * 128;        // 16 KB: 128 rows x 64 bf16 (SW128)
+constexpr int kUpStages = 6;
+constexpr int kUpStageBytes = 2 * kChunk;  // W chunk (two 64-feature halves) + c_KV chunk
+
+__device__ __forceinline__ void store_rows(uint32_t tmem, uint8_t* s_out, const CUtensorMap* tm_out, int h, int n0) {
+  // TMEM [128 lanes = features][128 columns = tokens] fp32 -> bf16 [token][128] -> one TMA store
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(s_out);
+  const int m = warp * 32 + lane;
+  for (int c = 0; c < kTile; c += 32) {
+    uint32_t r[32];
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[(c + j) * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    tma_store_3d(tm_out, s_out, 0, h, n0);
+    bulk_commit();
+    bulk_wait_all<0>();
+  }
+}
+
+struct UpParams {
+  const int32_t* block_row;   // the sequence's block-table row
+  int T, n_pages, num_blocks;
+};
+
+__global__ void __launch_bounds__(128)
+up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant__ CUtensorMap tm_wv,
+               const __grid_constant__ CUtensorMap tm_pool, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const UpParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kUpStages * kUpStageBytes);
+  uint64_t* empty = full + kUpStages;
+  uint64_t* done = empty + kUpStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const bool is_v = blockIdx.x == 1;
+  const int h = blockIdx.y, t0 = blockIdx.z * kTile;
+  const CUtensorMap* tm_w = is_v ? &tm_wv : &tm_wk;
+  constexpr int kChunks = 512 / 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kUpStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(tm_w);
+    prefetch_tmap(&tm_pool);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTile);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (warp == 0 && lane == 0) {
+    // block ids of the tile's two pages (pages past the sequence: block 0, clipped at the store)
+    int blk[2];
+    for (int q = 0; q < 2; ++q) {
+      const int pg = t0 / 64 + q;
+      int b = pg < p.n_pages ? p.block_row[pg] : 0;
+      blk[q] = (b < 0 || b >= p.num_blocks) ? 0 : b;
+    }
+    for (int kc = 0; kc < kChunks; ++kc) {
+      const int s = kc % kUpStages;
+      if (kc >= kUpStages && !mbar_wait(&empty[s], ((kc / kUpStages) - 1) & 1, abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      uint8_t* st = smem + s * kUpStageBytes;
+      mbar_arrive_expect_tx(&full[s], kUpStageBytes);
+      tma_load_3d(st, tm_w, &full[s], 0, h, kc * 64);                  // features 0..63 (MN-major)
+      tma_load_3d(st + kChunk / 2, tm_w, &full[s], 64, h, kc * 64);    // features 64..127
+      tma_load_3d(st + kChunk, &tm_pool, &full[s], kc * 64, 0, blk[0]);               // tokens 0..63
+      tma_load_3d(st + kChunk + kChunk / 2, &tm_pool, &full[s], kc * 64, 0, blk[1]);  // tokens 64..127
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_bf16(128, kTile, 1, 0);
+    for (int kc = 0; kc < kChunks; ++kc) {
+      const int s = kc % kUpStages;
+      if (!mbar_wait(&full[s], (kc / kUpStages) & 1, abort_flag)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(smem + s * kUpStageBytes), b0 = a0 + kChunk;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem, sdesc(a0 + kk * 2048, kChunk / 2, 1024, kSwizzle128B),
+               sdesc(b0 + kk * 32, 16, 1024, kSwizzle128B), idesc, (kc | kk) != 0);
+      mma_commit(&empty[s]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+  const bool ok = __syncthreads_and(mbar_wait(done, 0, abort_flag) && !*abort_flag);
+  tc_fence_after();
+  if (ok) store_rows(tmem, smem, is_v ? &tm_v : &tm_k, h, t0);
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  if (warp == 1) tmem_dealloc(tmem, kTile);
+}
+
+// ----------------------------------------------------------------- causal attention
+constexpr int kAttThreads = 224;            // 7 warps
+constexpr int kSoftWarp0 = 3;
+constexpr int kKStageBytes = 3 * kChunk;    // K (two 64-d chunks) + k_rope (one 64-col chunk)
+constexpr int kVStageBytes = 2 * kChunk;    // V as two 64-v chunks (MN-major B)
+constexpr int kStageBytes = kKStageBytes + kVStageBytes;   // 80 KB
+constexpr int kAttStages = 2;
+constexpr int kOffQ = 0;                                   // Q: q_nope (two chunks) + q_rope (one)
+constexpr int kOffStages = 3 * kChunk;
+constexpr int kOffBar = kOffStages + kAttStages * kStageBytes;
+constexpr uint32_t kTS = 0, kTP = 128, kTO = 256, kTCols = 512;
+constexpr float kRescale = 8.0f;            // log2 units
+
+struct AttBars {
+  uint64_t q_full, kv_full[kAttStages], kv_empty[kAttStages];
+  uint64_t s_full, s_read, p_full[2], o_full[2], o_done;
+  uint64_t qk_done, pv_done;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr int kAttSmem = kOffBar + (int)sizeof(AttBars) + 1024;
+
+struct AttParams {
+  const int32_t* block_row;
+  __nv_bfloat16* out;      // [s][H][128]
+  float* lse;              // [s][H] or null
+  int T, s, n_heads, n_pages, num_blocks;
+  float scale_log2;
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(kAttThreads, 1)
+prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qr,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_pool, const AttParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + kOffQ;
+  uint8_t* sKV = smem + kOffStages;
+  AttBars* bars = reinterpret_cast<AttBars*>(smem + kOffBar);
+  int* abort_flag = &bars->abort;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int qt = blockIdx.x, h = blockIdx.y;
+  const int q0 = qt * kTile;                              // first query of the tile (chunk index)
+  const int pos0 = p.T - p.s;                             // position of chunk query 0
+  const int last_q = min(q0 + kTile, p.s) - 1;
+  const int n_tiles = (pos0 + last_q) / kTile + 1;        // key tiles up to the causal limit
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kAttStages; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_read, 4);
+    mbar_init(&bars->p_full[0], 4);
+    mbar_init(&bars->p_full[1], 4);
+    mbar_init(&bars->o_full[0], 1);
+    mbar_init(&bars->o_full[1], 1);
+    mbar_init(&bars->o_done, 1);
+    mbar_init(&bars->qk_done, 1);
+    mbar_init(&bars->pv_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars->q_full, 3 * kChunk);
+      tma_load_3d(sQ, &tm_qn, &bars->q_full, 0, h, q0);             // rows past s: zero fill
+      tma_load_3d(sQ + kChunk, &tm_qn, &bars->q_full, 64, h, q0);
+      tma_load_3d(sQ + 2 * kChunk, &tm_qr, &bars->q_full, 0, h, q0);
+      int j = 0;
+      for (; j < n_tiles; ++j) {
+        const int s = j % kAttStages;
+        if (j >= kAttStages && !mbar_wait(&bars->kv_empty[s], ((j / kAttStages) - 1) & 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        int blk[2];
+        for (int q = 0; q < 2; ++q) {
+          const int pg = 2 * j + q;
+          const int b = pg < p.n_pages ? p.block_row[pg] : 0;
+          blk[q] = (b < 0 || b >= p.num_blocks) ? 0 : b;
+        }
+        uint8_t* st = sKV + s * kStageBytes;
+        mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
+        tma_load_3d(st, &tm_k, &bars->kv_full[s], 0, h, j * kTile);          // keys past T: zero fill
+        tma_load_3d(st + kChunk, &tm_k, &bars->kv_full[s], 64, h, j * kTile);
+        tma_load_3d(st + 2 * kChunk, &tm_pool, &bars->kv_full[s], 512, 0, blk[0]);   // k_rope, keys 0..63
+        tma_load_3d(st + 2 * kChunk + kChunk / 2, &tm_pool, &bars->kv_full[s], 512, 0, blk[1]);
+        tma_load_3d(st + kKStageBytes, &tm_v, &bars->kv_full[s], 0, h, j * kTile);
+        tma_load_3d(st + kKStageBytes + kChunk, &tm_v, &bars->kv_full[s], 64, h, j * kTile);
+      }
+      // every issued load must land before the CTA exits
+      for (int k = j - 1; k >= 0 && k >= j - kAttStages; --k)
+        mbar_drain(&bars->kv_full[k % kAttStages], (k / kAttStages) & 1);
+      mbar_drain(&bars->q_full, 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ QK issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, kTile, 0, 0);
+      bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
+      const uint32_t q_addr = smem_u32(sQ);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kAttStages;
+        if (!mbar_wait(&bars->kv_full[s], (j / kAttStages) & 1, abort_flag) ||
+            (j > 0 && !mbar_wait(&bars->s_read, (j - 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sKV + s * kStageBytes);
+#pragma unroll
+        for (int t = 0; t < 12; ++t) {   // K = 192 in steps of 16: chunk t / 4 (nope, nope, rope)
+          const uint32_t off = (t >> 2) * kChunk + (t & 3) * 32;
+          mma_ss(tmem + kTS, sdesc(q_addr + off, 16, 1024, kSwizzle128B), sdesc(k_addr + off, 16, 1024, kSwizzle128B),
+                 idesc, t != 0);
+        }
+        mma_commit(&bars->s_full);
+      }
+      if (!ok) *abort_flag = 1;
+      mma_commit(&bars->qk_done);
+      mbar_drain(&bars->qk_done, 0);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+      bool ok = true;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kAttStages;
+        if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sKV + s * kStageBytes + kKStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)   // 128 keys in steps of 16
+          mma_ts(tmem + kTO, tmem + kTP + 64 * (j & 1) + 8 * kk,
+                 sdesc(v_addr + kk * 2048, kChunk, 1024, kSwizzle128B), idesc, (j | kk) != 0);
+        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->o_full[j & 1]);
+      }
+      if (ok) mma_commit(&bars->o_done);
+      else *abort_flag = 1;
+      mma_commit(&bars->pv_done);
+      mbar_drain(&bars->pv_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (4 warps, one thread per query)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;                 // query row of the tile = TMEM lane
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const int qpos = pos0 + q0 + r;                    // position of this query (keys <= qpos visible)
+    const float sl2 = p.scale_log2;
+    float m_ref = -CUDART_INF_F, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t v[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + kTS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_read);
+      // causal mask: key j * 128 + c is visible iff <= qpos (which also excludes keys >= T)
+      const int vis = qpos - j * kTile;                // columns [0, vis] visible
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        float x = __uint_as_float(v[c]) * sl2;
+        if (c > vis) x = -CUDART_INF_F;
+        v[c] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      const bool move = (m_ref == -CUDART_INF_F) ? (m_new != -CUDART_INF_F) : (m_new > m_ref + kRescale);
+      float alpha = 1.f;
+      if (move) {
+        alpha = (m_ref == -CUDART_INF_F) ? 0.f : ex2f(m_ref - m_new);
+        m_ref = m_new;
+      }
+      const float nb = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+      uint32_t pk[64];
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 64; ++k) {
+        const float e0 = ex2f(__uint_as_float(v[2 * k]) + nb), e1 = ex2f(__uint_as_float(v[2 * k + 1]) + nb);
+        pk[k] = pack_bf16(e0, e1);
+        ps[k & 3] += e0 + e1;
+      }
+      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      // P buffer j & 1 is free once the PV product of tile j - 2 completed
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->o_full[j & 1], ((j >> 1) - 1) & 1, abort_flag))) {
+        ok = false;
+        break;
+      }
+      if (__any_sync(0xffffffffu, move && j > 0)) {
+        // rescale O: the PV product of tile j - 1 must have landed
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float a = (move && j > 0) ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_addr + kTO + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+          tmem_st32(tmem + lane_addr + kTO + 32 * c, o);
+        }
+        tmem_st_wait();
+      }
+      tmem_st32(tmem + lane_addr + kTP + 64 * (j & 1), *reinterpret_cast<uint32_t(*)[32]>(pk));
+      tmem_st32(tmem + lane_addr + kTP + 64 * (j & 1) + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[j & 1]);
+    }
+    if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_done, 0, abort_flag))) ok = false;
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const int q = q0 + r;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_addr + kTO + 32 * c, o);
+        tmem_ld_wait();
+        if (q < p.s) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)q * p.n_heads + h) * 128 + 32 * c);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(pack_bf16(__uint_as_float(o[8 * k]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
+                                pack_bf16(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
+                                pack_bf16(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
+                                pack_bf16(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+        }
+      }
+      if (q < p.s && p.lse) p.lse[(size_t)q * p.n_heads + h] = l_run > 0.f ? (m_ref + __log2f(l_run)) * 0.6931471805599453f : -CUDART_INF_F;
+    } else {
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  if (warp == 1) tmem_dealloc(tmem, kTCols);
+}
+
+cudaError_t prefill_attrs() {
+  static cudaError_t e = [] {
+    cudaError_t a = cudaFuncSetAttribute(up_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         1024 + kUpStages * kUpStageBytes + 256);
+    cudaError_t b = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
+    return a != cudaSuccess ? a : b;
+  }();
+  return e;
+}
+
+// [N][H][F] bf16 viewed as (F, H, N): boxes of 64 features x 128 rows (SW128), or a
+// store box of 128 features x 128 rows (no swizzle).
+mla_status_t rows_map(CUtensorMap* m, const void* base, int F, int H, int N, bool store) {
+  const uint64_t dims[3] = {(uint64_t)F, (uint64_t)H, (uint64_t)N};
+  const uint64_t str[2] = {(uint64_t)F * 2, (uint64_t)H * F * 2};
+  const uint32_t box[3] = {store ? 128u : 64u, 1, (uint32_t)kTile};
+  return encode_tmap_bf16(m, base, 3, dims, str, box, store ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// The cache pool as (column, row within the block, block), boxes of 64 columns x 64 rows.
+mla_status_t pool_map(CUtensorMap* m, const void* pool, int num_blocks) {
+  const uint64_t dims[3] = {576, 64, (uint64_t)num_blocks};
+  const uint64_t str[2] = {576 * 2, 64 * 576 * 2};
+  const uint32_t box[3] = {64, 64, 1};
+  return encode_tmap_bf16(m, pool, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+mla_status_t launch_prefill_up_proj(const void* kv_pool, const int32_t* block_row, int T, int num_blocks,
+                                    const void* w_uk, const void* w_uv, int n_heads, void* k_out, void* v_out,
+                                    void* stream) {
+  CUtensorMap twk, twv, tpool, tk, tv;
+  const uint64_t wdims[3] = {128, (uint64_t)n_heads, 512};
+  const uint64_t wstr[2] = {128 * 2, (uint64_t)n_heads * 128 * 2};
+  const uint32_t wbox[3] = {64, 1, 64};
+  mla_status_t st = encode_tmap_bf16(&twk, w_uk, 3, wdims, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st == MLA_OK) st = encode_tmap_bf16(&twv, w_uv, 3, wdims, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st == MLA_OK) st = pool_map(&tpool, kv_pool, num_blocks);
+  if (st == MLA_OK) st = rows_map(&tk, k_out, 128, n_heads, T, true);
+  if (st == MLA_OK) st = rows_map(&tv, v_out, 128, n_heads, T, true);
+  if (st != MLA_OK) return st;
+  UpParams p{block_row, T, (T + 63) / 64, num_blocks};
+  cudaError_t e = prefill_attrs();
+  if (e == cudaSuccess) {
+    e = launch_pdl(up_proj_kernel, dim3(2, n_heads, (T + kTile - 1) / kTile), dim3(128),
+                   1024 + kUpStages * kUpStageBytes + 256, stream, twk, twv, tpool, tk, tv, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "prefill up-projection launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_prefill_attn(const void* q_nope, const void* q_rope, const void* k, const void* v,
+                                 const void* kv_pool, const int32_t* block_row, int T, int s, int n_heads,
+                                 int num_blocks, float scale, void* out, float* lse, void* stream) {
+  CUtensorMap tqn, tqr, tk, tv, tpool;
+  mla_status_t st = rows_map(&tqn, q_nope, 128, n_heads, s, false);
+  if (st == MLA_OK) st = rows_map(&tqr, q_rope, 64, n_heads, s, false);
+  if (st == MLA_OK) st = rows_map(&tk, k, 128, n_heads, T, false);
+  if (st == MLA_OK) st = rows_map(&tv, v, 128, n_heads, T, false);
+  if (st == MLA_OK) st = pool_map(&tpool, kv_pool, num_blocks);
+  if (st != MLA_OK) return st;
+  AttParams p{block_row, static_cast<__nv_bfloat16*>(out), lse, T, s, n_heads, (T + 63) / 64, num_blocks,
+              scale * 1.4426950408889634f};
+  cudaError_t e = prefill_attrs();
+  if (e == cudaSuccess) {
+    e = launch_pdl(prefill_attn_kernel, dim3((s + kTile - 1) / kTile, n_heads), dim3(kAttThreads), kAttSmem, stream,
+                   tqn, tqr, tk, tv, tpool, p);
+    if (e == cudaSuccess) e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "prefill attention launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+}  // namespace mla

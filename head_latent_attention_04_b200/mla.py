@@ -28,7 +28,8 @@ EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
            "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes",
            "mla_quantize_w_uk_fp8", "mla_quantize_w_uv_fp8", "mla_quantize_rows_fp8", "mla_absorb_q_fp8",
-           "mla_out_uv_fp8", "mla_set_wait_limit_ns", "mla_decode_attn_tree")
+           "mla_out_uv_fp8", "mla_set_wait_limit_ns", "mla_decode_attn_tree", "mla_prefill_up_proj",
+           "mla_prefill_attn")
 
 
 class MlaDims(ctypes.Structure):
@@ -59,6 +60,8 @@ for _name, _args in {
     "mla_quantize_rows_fp8": [_vp, ctypes.c_int64, _i32, _vp, _vp, _vp],
     "mla_absorb_q_fp8": [_vp, _vp, _vp, _vp, _i32, _i32, _vp],
     "mla_out_uv_fp8": [_vp, _vp, _vp, _vp, _i32, _i32, _vp],
+    "mla_prefill_up_proj": [_vp, _vp, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp],
+    "mla_prefill_attn": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_float, _vp, _vp, _vp],
 }.items():
     getattr(_lib, _name).argtypes = _args
     getattr(_lib, _name).restype = _i32
@@ -238,6 +241,37 @@ def decode_attn_tree(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_
 def combine(dims, plan_dev, o_part, lse_part, o_lat, lse_out=None, stream=None):
     _check(_lib.mla_combine(ctypes.byref(dims), _ptr(plan_dev), _ptr(o_part), _ptr(lse_part),
                             _ptr(o_lat), _ptr(lse_out), _stream(stream)), "mla_combine")
+
+
+def prefill_up_proj(kv_pool, block_row, T, w_uk, w_uv, k_out=None, v_out=None, stream=None):
+    """K and V [T][h][128] of one sequence's first T cached tokens (order 1)."""
+    H = w_uk.shape[1]
+    if k_out is None:
+        k_out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=kv_pool.device)
+    if v_out is None:
+        v_out = torch.empty((T, H, 128), dtype=torch.bfloat16, device=kv_pool.device)
+    _check(_lib.mla_prefill_up_proj(_ptr(kv_pool), _ptr(block_row), T, kv_pool.shape[0], _ptr(w_uk), _ptr(w_uv), H,
+                                    _ptr(k_out), _ptr(v_out), _stream(stream)), "mla_prefill_up_proj")
+    return k_out, v_out
+
+
+def prefill_attn(q_nope, q_rope, k, v, kv_pool, block_row, T, scale=None, out=None, lse=None, stream=None):
+    """Causal attention of the last s = q_nope.shape[0] of T cached tokens."""
+    s, H, _ = q_nope.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(128 + 64)
+    if out is None:
+        out = torch.empty((s, H, 128), dtype=torch.bfloat16, device=q_nope.device)
+    _check(_lib.mla_prefill_attn(_ptr(q_nope), _ptr(q_rope), _ptr(k), _ptr(v), _ptr(kv_pool), _ptr(block_row), T, s,
+                                 H, kv_pool.shape[0], float(scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "mla_prefill_attn")
+    return out
+
+
+def prefill(q_nope, q_rope, kv_pool, block_row, T, w_uk, w_uv, scale=None, lse=None, stream=None):
+    """Prefill (s = T) or a prefill chunk (s < T) of one sequence in order 1."""
+    k, v = prefill_up_proj(kv_pool, block_row, T, w_uk, w_uv, stream=stream)
+    return prefill_attn(q_nope, q_rope, k, v, kv_pool, block_row, T, scale=scale, lse=lse, stream=stream)
 
 
 def noalloc_scratch_bytes() -> int:

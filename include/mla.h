@@ -283,6 +283,38 @@ mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void*
                                              int32_t num_clusters, void* o_lat, float* lse_out,
                                              int32_t* status, void* stream);
 
+/*
+ * Prefill and chunked prefill in order 1 ("MHA form").  "MLA Matrix
+ * Absorption Analysis" section 2.4.1: when the query length equals the key
+ * length (t = s) the un-absorbed order 1 needs fewer FLOPs than the absorbed
+ * order 2 (by 98304 s^2 at DeepSeek-V3 widths), and the Perplexity write-up's
+ * future-work section names prefill in the up-projected form and chunked
+ * prefill.  One sequence per call; its cache rows are read through its
+ * block-table row (int32 [ceil(T / 64)], device), as in decode.
+ *
+ * mla_prefill_up_proj -- K and V of the sequence's first T tokens:
+ *   K[t,h,:] = W_UK[:,h,:]^T c_KV[t]   (notes section 2.1 Step 2)
+ *   V[t,h,:] = W_UV[:,h,:]^T c_KV[t]   (notes section 3.1 Step 1)
+ *   k_out, v_out   bf16 [T][n_heads][128] (device, written; fp32 accumulation)
+ *   w_uk, w_uv     bf16 [512][n_heads][128]
+ *
+ * mla_prefill_attn -- causal attention of the chunk's s query tokens (the last
+ * s of the T cached tokens, positions T - s .. T - 1; s = T is a full
+ * prefill, s < T a chunk after a prefix) over K, V and the cached RoPE keys:
+ *   logit[i,h,t] = scale (q_nope[i,h] . K[t,h] + q_rope[i,h] . k_rope[t])
+ *   out[i,h,:]   = sum_{t <= T - s + i} softmax_t(logit) V[t,h,:]
+ *   q_nope bf16 [s][n_heads][128], q_rope bf16 [s][n_heads][64] (post-rotation)
+ *   k, v   bf16 [T][n_heads][128] from mla_prefill_up_proj
+ *   out    bf16 [s][n_heads][128] (written), lse fp32 [s][n_heads] or NULL
+ * 1 <= s <= T <= 2^22, 1 <= n_heads <= 128.
+ */
+mla_status_t mla_prefill_up_proj(const void* kv_pool, const int32_t* block_table_row, int32_t T, int32_t num_blocks,
+                                 const void* w_uk, const void* w_uv, int32_t n_heads, void* k_out, void* v_out,
+                                 void* stream);
+mla_status_t mla_prefill_attn(const void* q_nope, const void* q_rope, const void* k, const void* v,
+                              const void* kv_pool, const int32_t* block_table_row, int32_t T, int32_t s,
+                              int32_t n_heads, int32_t num_blocks, float scale, void* out, float* lse, void* stream);
+
 /* Size in bytes of the device array mla_decode_attn_combine_noalloc works in. */
 size_t mla_noalloc_scratch_bytes(void);
 

@@ -159,7 +159,7 @@ def test_decode_order1_equals_absorbed(s_q, lens):
     np.testing.assert_allclose(ref["q_lat"], ql, rtol=1e-12, atol=1e-12)
 
 
-@pytest.mark.parametrize("s_q,T", [(1, 1), (1, 3), (1, 5), (2, 3), (2, 5), (2, 2)])
+@pytest.mark.parametrize("s_q,T", [(1, 1), (1, 3), (1, 5), (2, 3), (2, 5), (2, 2), (4, 4), (3, 5)])
 def test_decode_matches_brute_force(s_q, T):
     rng = np.random.default_rng(10 + T + s_q)
     B, H, d, R, k, v = 2, 2, 4, 2, 8, 4
