@@ -178,6 +178,30 @@ def second_absorption_output(order: int, score, ckv, W_UV, W_O=None, counter=Non
     return out
 
 
+def query_up(c_q, W_UQ, d_nope: int = D_NOPE, counter=None):
+    """Per-head queries from the query latent: q = W^UQ applied to c^Q.
+
+    ``c_q`` (n, q) and ``W_UQ`` (q, h, d + R), the notes' W^UQ (q, h, d) of
+    section 2.1 extended by the head's RoPE query columns (DeepSeek's q_b_proj
+    produces both).  Returns (q_nope (n, h, d), q_rope (n, h, R)); the RoPE
+    part is returned before rotation.  Label 'uq' (2 n q h (d + R)).
+    """
+    q = contract(counter, "uq", "nq,qhf->nhf", c_q, W_UQ)
+    if isinstance(q, Shape):   # dry run: shapes only
+        n, h, f = q.shape
+        return Shape((n, h, d_nope)), Shape((n, h, f - d_nope))
+    return q[:, :, :d_nope], q[:, :, d_nope:]
+
+
+def qkv_down(x, W_DQ, W_DKV, counter=None):
+    """The two down-projections of a token's hidden state, as the Perplexity
+    write-up's fused qkv_a_proj computes them in one product (section "MLA
+    layer": q_a_proj and kv_a_proj merged): c^Q = x W^DQ (n, q) and the
+    cache row [c^KV | k_rope] = x W^DKV (n, d_c + R), k_rope before rotation.
+    ``x`` (n, e), ``W_DQ`` (e, q), ``W_DKV`` (e, d_c + R).  Labels 'dq', 'dkv'."""
+    return contract(counter, "dq", "ne,eq->nq", x, W_DQ), contract(counter, "dkv", "ne,ec->nc", x, W_DKV)
+
+
 def rope_logits(q_rope, k_rope, counter=None):
     """Decoupled-RoPE score q_rope . k_rope, (b,h,s,t); one key shared by all heads.
 
