@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmla.so")
-SOURCES = ["capi.cu", "plan.cpp", "head_gemm.cu", "decode_attn.cu", "combine.cu", "noalloc.cu", "prefill.cu"]
+SOURCES = ["capi.cu", "plan.cpp", "head_gemm.cu", "decode_attn.cu", "combine.cu", "noalloc.cu", "prefill.cu", "upstream.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -309,6 +309,29 @@ mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void*
 
 size_t mla_noalloc_scratch_bytes(void) { return noalloc_scratch_bytes(); }
 
+mla_status_t mla_q_up_absorb(const void* c_q, const void* w_uq, const void* w_uk, void* q_lat, void* q_rope,
+                             int32_t n_tokens, int32_t n_heads, void* stream) {
+  clear_error();
+  MLA_TRY(check_tokens(n_tokens, n_heads));
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(w_uq, "w_uq"));
+  MLA_TRY(check_ptr(w_uk, "w_uk"));
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  MLA_TRY(check_ptr(q_rope, "q_rope"));
+  return launch_q_up_absorb(c_q, w_uq, w_uk, q_lat, q_rope, n_tokens, n_heads, stream);
+}
+
+mla_status_t mla_qkv_a_proj(const void* x, const void* w_qkv_a, void* c_q, void* kv_a, int32_t n_tokens,
+                            void* stream) {
+  clear_error();
+  if (n_tokens < 1 || n_tokens > 65536) return set_error(MLA_ERR_UNSUPPORTED, "n_tokens must be in [1, 65536]");
+  MLA_TRY(check_ptr(x, "x"));
+  MLA_TRY(check_ptr(w_qkv_a, "w_qkv_a"));
+  MLA_TRY(check_ptr(c_q, "c_q"));
+  MLA_TRY(check_ptr(kv_a, "kv_a"));
+  return launch_qkv_a_proj(x, w_qkv_a, c_q, kv_a, n_tokens, stream);
+}
+
 static mla_status_t check_prefill(int T, int s, int n_heads, int num_blocks) {
   if (n_heads < 1 || n_heads > 128) return set_error(MLA_ERR_UNSUPPORTED, "n_heads must be in [1, 128]");
   if (T < 1 || T > (1 << 22)) return set_error(MLA_ERR_UNSUPPORTED, "T must be in [1, 2^22]");

@@ -63,6 +63,9 @@ mla_status_t launch_prefill_up_proj(const void* kv_pool, const int32_t* block_ro
 mla_status_t launch_prefill_attn(const void* q_nope, const void* q_rope, const void* k, const void* v,
                                  const void* kv_pool, const int32_t* block_row, int T, int s, int n_heads,
                                  int num_blocks, float scale, void* out, float* lse, void* stream);
+mla_status_t launch_q_up_absorb(const void* c_q, const void* w_uq, const void* w_uk, void* q_lat, void* q_rope,
+                                int n_tokens, int n_heads, void* stream);
+mla_status_t launch_qkv_a_proj(const void* x, const void* w, void* c_q, void* kv_a, int n_tokens, void* stream);
 mla_status_t launch_gather_pages(const void* kv_pool, const int32_t* block_table, int32_t b,
                                  int32_t n_pages, int32_t max_blocks, int32_t num_blocks, void* out,
                                  int32_t* status, void* stream);

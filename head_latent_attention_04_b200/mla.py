@@ -29,7 +29,7 @@ EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes",
            "mla_quantize_w_uk_fp8", "mla_quantize_w_uv_fp8", "mla_quantize_rows_fp8", "mla_absorb_q_fp8",
            "mla_out_uv_fp8", "mla_set_wait_limit_ns", "mla_decode_attn_tree", "mla_prefill_up_proj",
-           "mla_prefill_attn")
+           "mla_prefill_attn", "mla_qkv_a_proj", "mla_q_up_absorb")
 
 
 class MlaDims(ctypes.Structure):
@@ -61,6 +61,8 @@ for _name, _args in {
     "mla_absorb_q_fp8": [_vp, _vp, _vp, _vp, _i32, _i32, _vp],
     "mla_out_uv_fp8": [_vp, _vp, _vp, _vp, _i32, _i32, _vp],
     "mla_prefill_up_proj": [_vp, _vp, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _vp],
+    "mla_qkv_a_proj": [_vp, _vp, _vp, _vp, _i32, _vp],
+    "mla_q_up_absorb": [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp],
     "mla_prefill_attn": [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_float, _vp, _vp, _vp],
 }.items():
     getattr(_lib, _name).argtypes = _args
@@ -241,6 +243,29 @@ def decode_attn_tree(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_
 def combine(dims, plan_dev, o_part, lse_part, o_lat, lse_out=None, stream=None):
     _check(_lib.mla_combine(ctypes.byref(dims), _ptr(plan_dev), _ptr(o_part), _ptr(lse_part),
                             _ptr(o_lat), _ptr(lse_out), _stream(stream)), "mla_combine")
+
+
+def qkv_a_proj(x, w_qkv_a, c_q=None, kv_a=None, stream=None):
+    """Fused down-projections: x [N][7168] -> c_q [N][1536], kv_a [N][576]."""
+    N = x.shape[0]
+    if c_q is None:
+        c_q = torch.empty((N, 1536), dtype=torch.bfloat16, device=x.device)
+    if kv_a is None:
+        kv_a = torch.empty((N, 576), dtype=torch.bfloat16, device=x.device)
+    _check(_lib.mla_qkv_a_proj(_ptr(x), _ptr(w_qkv_a), _ptr(c_q), _ptr(kv_a), N, _stream(stream)), "mla_qkv_a_proj")
+    return c_q, kv_a
+
+
+def q_up_absorb(c_q, w_uq, w_uk, q_lat=None, q_rope=None, stream=None):
+    """c_q [N][1536] -> q_lat [N][h][512] (through W_UQ then W_UK) and q_rope [N][h][64]."""
+    N, H = c_q.shape[0], w_uq.shape[1]
+    if q_lat is None:
+        q_lat = torch.empty((N, H, 512), dtype=torch.bfloat16, device=c_q.device)
+    if q_rope is None:
+        q_rope = torch.empty((N, H, 64), dtype=torch.bfloat16, device=c_q.device)
+    _check(_lib.mla_q_up_absorb(_ptr(c_q), _ptr(w_uq), _ptr(w_uk), _ptr(q_lat), _ptr(q_rope), N, H, _stream(stream)),
+           "mla_q_up_absorb")
+    return q_lat, q_rope
 
 
 def prefill_up_proj(kv_pool, block_row, T, w_uk, w_uv, k_out=None, v_out=None, stream=None):

@@ -284,6 +284,32 @@ mla_status_t mla_decode_attn_combine_noalloc(const mla_dims_t* dims, const void*
                                              int32_t* status, void* stream);
 
 /*
+ * Upstream of the absorbed path, fused.
+ *
+ * mla_qkv_a_proj -- the Perplexity write-up's qkv_a_proj ("MLA layer": q_a_proj
+ * and kv_a_proj merged into one product): for the hidden states of N tokens,
+ *   c_q  = x W^DQ   and   kv_a = x W^DKV = [c_KV | k_rope (before rotation)]
+ *   x        bf16 [N][7168]           (DeepSeek-V3 model width)
+ *   w_qkv_a  bf16 [2112][7168]        rows 0..1535 = W^DQ^T, rows 1536..2111 = W^DKV^T
+ *   c_q      bf16 [N][1536] (written), kv_a bf16 [N][576] (written; the cache row)
+ * fp32 accumulation; one launch (the K range is split over a cluster of 8
+ * CTAs and reduced through distributed shared memory).  1 <= N <= 65536.
+ *
+ * mla_q_up_absorb -- the query up-projection feeding the first absorption
+ * without q_nope leaving the SM ("MLA Matrix Absorption Analysis" section 2.2
+ * Steps 1-2, terms 2bshdq and 2bshkd):
+ *   q[n,h,:]     = sum_j c_q[n,j] W_UQ[j,h,:]           (128 nope + 64 RoPE columns)
+ *   q_lat[n,h,:] = sum_d q[n,h,d] W_UK[:,h,d]            (d < 128)
+ *   c_q    bf16 [N][1536], w_uq bf16 [1536][n_heads][192] (q, h, d + R), w_uk bf16 [512][n_heads][128]
+ *   q_lat  bf16 [N][n_heads][512] (written), q_rope bf16 [N][n_heads][64] (written, before rotation)
+ * W_UQ^T W_UK is never formed.  1 <= N <= 65536, 1 <= n_heads <= 128.
+ */
+mla_status_t mla_qkv_a_proj(const void* x, const void* w_qkv_a, void* c_q, void* kv_a, int32_t n_tokens,
+                            void* stream);
+mla_status_t mla_q_up_absorb(const void* c_q, const void* w_uq, const void* w_uk, void* q_lat, void* q_rope,
+                             int32_t n_tokens, int32_t n_heads, void* stream);
+
+/*
  * Prefill and chunked prefill in order 1 ("MHA form").  "MLA Matrix
  * Absorption Analysis" section 2.4.1: when the query length equals the key
  * length (t = s) the un-absorbed order 1 needs fewer FLOPs than the absorbed
