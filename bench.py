@@ -62,24 +62,28 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--projections", default="bf16", choices=["bf16", "fp8"],
                     help="absorb / out_uv as bf16 GEMMs or as FP8 (E4M3) block-quantised BMMs")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"],
+                    help="latent cache rows as bf16 (1152 B/token) or E4M3 codes with fp32 block scales "
+                         "and a bf16 k_rope (656 B/token)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------------------- accounting
-def algorithmic(seq_lens, s_q, H, causal=True, weight_bytes=2):
+def algorithmic(seq_lens, s_q, H, causal=True, weight_bytes=2, cache_row_bytes=1152):
     """Algorithmic bytes / FLOPs of the step and of the attention kernel.
 
     Per attended (query, key) pair: 2*h*(2*d_c + d_R) FLOPs (QK over 576 +
-    PV over 512 per head).  Per cached token: 576 bf16 = 1152 B, read once
-    and shared by all heads and all s_q query tokens of its sequence.
+    PV over 512 per head).  Per cached token: one cache row, read once and
+    shared by all heads and all s_q query tokens of its sequence: 576 bf16 =
+    1152 B, or 656 B for the FP8 cache (512 E4M3 codes, 4 fp32 scales, 64 bf16).
     ``weight_bytes``: bytes per W_UK / W_UV element (1 for E4M3 codes, whose
     scales add 4 bytes per 128 x 128 block).
     """
     T = np.asarray(seq_lens, dtype=np.int64)
     N = len(T) * s_q
     pairs = int(sum(int(t) - s_q + 1 + i if causal else int(t) for t in T for i in range(s_q)))
-    cache = int(T.sum()) * 576 * 2
+    cache = int(T.sum()) * cache_row_bytes
     w_bytes = 2 * 512 * H * 128 * weight_bytes + (2 * 4 * H * 4 if weight_bytes == 1 else 0)
     attn_flops = pairs * 2 * H * (2 * 512 + 64)
     bmm_flops = 2 * (2 * N * H * 128 * 512)
@@ -314,16 +318,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     preset = W.PRESETS[args.config]
     w = W.preset_workload(args.config, device=dev, seed=dp.replica_seed(preset.seed, rank))
     fp8 = args.projections == "fp8"
-    acc = algorithmic(w.seq_lens, w.s_q, w.n_heads, weight_bytes=1 if fp8 else 2)
+    fp8_cache = args.cache == "fp8"
+    acc = algorithmic(w.seq_lens, w.s_q, w.n_heads, weight_bytes=1 if fp8 else 2,
+                      cache_row_bytes=mla.FP8_ROW_BYTES if fp8_cache else 1152)
     bt = torch.as_tensor(w.block_table, device=dev)
-    dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev)
+    dec = mla.Decoder(w.seq_lens, w.s_q, w.n_heads, w.max_blocks, w.num_blocks, dev, kv_cache=args.cache)
     if fp8:   # weights quantised once, outside the timed region (static, as the weights are)
         dec.use_fp8_projections(w.w_uk, w.w_uv)
+    if fp8_cache:   # the cache written once in FP8 (as a serving loop writes each new row), then resident
+        pool = mla.fp8_pool_from(w.kv_pool)
+        torch.cuda.synchronize()
+    else:
+        pool = w.kv_pool
+    attn_fn = mla.decode_attn_fp8cache if fp8_cache else mla.decode_attn
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        dec.run(w.q_nope, w.q_rope, w.kv_pool, bt, w.w_uk, w.w_uv)
+        dec.run(w.q_nope, w.q_rope, pool, bt, w.w_uk, w.w_uv)
 
     for _ in range(max(args.warmup, 3)):
         flush.zero_()
@@ -369,8 +381,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         for i in range(K):
             flush.zero_()
             ea[i][0].record(stream)
-            mla.decode_attn(dec.dims, dec.q_lat, w.q_rope, w.kv_pool, bt, dec.seq_lens_dev, dec.plan_dev,
-                            dec.num_clusters, dec.o_part, dec.lse_part, dec.o_lat, dec.lse, dec.status)
+            attn_fn(dec.dims, dec.q_lat, w.q_rope, pool, bt, dec.seq_lens_dev, dec.plan_dev,
+                    dec.num_clusters, dec.o_part, dec.lse_part, dec.o_lat, dec.lse, dec.status)
             ea[i][1].record(stream)
         barrier()
     t_wall = time.perf_counter() - t_wall
@@ -386,7 +398,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # Serial (latency): mla.GraphedStep replays one graph per step (pinned H2D of
     # the queries and page table, the four kernels, D2H of the output), with L2
     # flushed before every step outside the events.
-    gs = mla.GraphedStep(dec, w.kv_pool, w.w_uk, w.w_uv)
+    gs = mla.GraphedStep(dec, pool, w.w_uk, w.w_uv)
     gs.q_nope.copy_(w.q_nope.cpu())
     gs.q_rope.copy_(w.q_rope.cpu())
     gs.block_table.copy_(torch.as_tensor(w.block_table))
@@ -408,7 +420,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # its neighbours' kernels; K back-to-back steps timed as one region.  No
     # flush inside the region: every step streams the whole KV cache, which is
     # larger than L2 for the full-size workloads.
-    sd = mla.StreamedDecoder(dec, w.kv_pool, w.w_uk, w.w_uv)
+    sd = mla.StreamedDecoder(dec, pool, w.w_uk, w.w_uv)
     for qn_h, qr_h, bt_h in sd.host_in:
         qn_h.copy_(w.q_nope.cpu())
         qr_h.copy_(w.q_rope.cpu())
@@ -446,7 +458,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         achieved = acc["attn_bytes"] / (attn * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-    roof.update({"traffic": recorded_traffic(args.config), "kernel": "mla_decode_kernel",
+    roof.update({"traffic": recorded_traffic(args.config + ("_fp8cache" if fp8_cache else "")),
+                 "kernel": "mla_decode_kernel" + ("<fp8 cache>" if fp8_cache else ""),
                  "alg_bytes_per_launch": acc["attn_bytes"], "alg_flops_per_launch": acc["attn_flops"],
                  "kernel_ms": attn, "peak_source": f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'}, burst)"})
     step_roof_s = max(acc["step_bytes"] / (peaks["hbm_gbs"] * 1e9), acc["step_flops"] / (peaks["bf16_tflops"] * 1e12))
@@ -455,11 +468,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "metric": METRIC, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 (attention); e4m3 codes with fp32 block scales (projections)" if fp8 else "bf16",
+        "dtype": ("bf16 (attention" + ("; the latent cache stored as e4m3 codes with fp32 block scales, "
+                                       "widened to bf16 on chip" if fp8_cache else "") + ")"
+                  + ("; e4m3 codes with fp32 block scales (projections)" if fp8 else "")) if (fp8 or fp8_cache)
+                 else "bf16",
         "data": "synthetic",
         "config": dict(workload_config(args.config, w), parallelism=f"dp{world} (independent replicas)",
                        num_clusters=dec.num_clusters, split_slots=dec.num_slots,
-                       graph=used_graph, projections=args.projections),
+                       graph=used_graph, projections=args.projections, kv_cache=args.cache),
         "cache_tbs": acc["cache_bytes"] * world / (ms * 1e-3) / 1e12,
         "attn_cache_tbs": acc["cache_bytes"] / (attn * 1e-3) / 1e12,
         "tflops": acc["step_flops"] * world / (ms * 1e-3) / 1e12,

@@ -275,6 +275,40 @@ mla_status_t mla_decode_attn_tree(const mla_dims_t* dims, const void* q_lat, con
                             o_lat, lse_out, status, stream);
 }
 
+mla_status_t mla_decode_attn_fp8cache(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                                      const void* kv_pool_fp8, const int32_t* block_table,
+                                      const int32_t* seq_lens, const void* plan_dev, int32_t num_clusters,
+                                      float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                                      int32_t* status, void* stream) {
+  clear_error();
+  MLA_TRY(check_dims(dims));
+  MLA_TRY(check_ptr(q_lat, "q_lat"));
+  MLA_TRY(check_ptr(q_rope, "q_rope"));
+  MLA_TRY(check_ptr(kv_pool_fp8, "kv_pool_fp8"));
+  MLA_TRY(check_ptr(block_table, "block_table"));
+  MLA_TRY(check_ptr(seq_lens, "seq_lens"));
+  MLA_TRY(check_ptr(plan_dev, "plan_dev"));
+  MLA_TRY(check_ptr(o_lat, "o_lat"));
+  if (num_clusters < 1 || num_clusters > 4096)
+    return set_error(MLA_ERR_INVALID_ARG, "num_clusters must be in [1, 4096]");
+  if ((o_part && (reinterpret_cast<uintptr_t>(o_part) & 31u)) || (lse_part && (reinterpret_cast<uintptr_t>(lse_part) & 3u)))
+    return set_error(MLA_ERR_INVALID_ARG, "o_part must be 32-byte aligned, lse_part 4-byte aligned");
+  return launch_decode_attn_fp8cache(*dims, q_lat, q_rope, kv_pool_fp8, block_table, seq_lens,
+                                     static_cast<const int32_t*>(plan_dev), num_clusters, o_part, lse_part,
+                                     o_lat, lse_out, status, stream);
+}
+
+mla_status_t mla_kv_quantize_fp8(const void* kv, const int32_t* slots, int64_t n, void* pool_fp8,
+                                 int32_t num_blocks, int32_t* status, void* stream) {
+  clear_error();
+  if (n < 0 || num_blocks < 1) return set_error(MLA_ERR_INVALID_ARG, "n must be >= 0 and num_blocks >= 1");
+  if (n == 0) return MLA_OK;
+  MLA_TRY(check_ptr(kv, "kv"));
+  MLA_TRY(check_ptr(slots, "slots"));
+  MLA_TRY(check_ptr(pool_fp8, "pool_fp8"));
+  return launch_kv_quantize_fp8(kv, slots, n, pool_fp8, (long long)num_blocks * 64, status, stream);
+}
+
 mla_status_t mla_combine(const mla_dims_t* dims, const void* plan_dev, const float* o_part,
                          const float* lse_part, void* o_lat, float* lse_out, void* stream) {
   clear_error();

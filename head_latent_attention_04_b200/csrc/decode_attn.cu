@@ -42,6 +42,19 @@
 // items the host plan gives it.  Every wait is bounded (200 ms by default,
 // mla_set_wait_limit_ns); on expiry the CTA sets MLA_STATUS_TIMEOUT, stops its
 // peer, drains the copies and products it issued and returns without trapping.
+//
+// FP8 latent cache (mla_decode_attn_fp8cache).  A token row is then 656
+// bytes: c_KV as 512 E4M3 codes, one fp32 scale per 128-column block, and
+// k_rope in bf16 (the block scheme of "Lower latency and higher throughput
+// with multi-node DeepSeek deployment", section "Quantization", applied to
+// the cached activation).  The producer loads a CTA's two code blocks, their
+// scales and its RoPE columns raw (21 KB of HBM per half page instead of
+// 36 KB), and the four sender warps widen the stage in place to the layout
+// above in fp16 (code x scale, one fp16 multiply per pair of codes: two
+// instructions per pair, where a bf16 result would take six), two pages ahead
+// of the QK product.  The latent products then run as kind::f16 with fp16
+// operands: q_lat is rounded to fp16 when it is loaded, P is written as fp16
+// pairs; the RoPE products stay bf16.  Everything else is the bf16 kernel.
 #include "mla_internal.h"
 #include "plan_format.h"
 #include "ptx.cuh"
@@ -63,6 +76,13 @@ constexpr int kStages = 5;
 constexpr int kChunkBytes = kPage * 128;                     // 64 keys x 64 latent cols (SW128)
 constexpr int kRopeBytes = kPage * 64;                       // 64 keys x 32 rope cols (SW64)
 constexpr int kStageBytes = 4 * kChunkBytes + kRopeBytes;    // 36 KB: half a page
+// FP8 cache row: [512 E4M3 codes | 4 fp32 scales | 64 bf16 k_rope].  Raw stage
+// layout: code block h of this CTA (128 bytes per key, SW128) in chunk 2h + 1;
+// the scales of keys [16w, 16w + 16) (16 bytes each) at 2048 w, inside the rows
+// of chunk 0 that sender warp w alone rewrites; RoPE where the bf16 stage has it.
+constexpr int kF8Row = 656, kF8ScaleOff = 512, kF8RopeOff = 528;
+constexpr int kF8ScaleKeys = 16;
+constexpr int kF8StageTx = 2 * kChunkBytes + (kPage / kF8ScaleKeys) * kF8ScaleKeys * 16 + kRopeBytes;
 constexpr int kXRow = 64 * 2;                                // fp16 score row, 16B chunks XOR (row & 7)
 constexpr int kXBytes = kRows * kXRow;                       // one score tile (16 KB)
 
@@ -101,6 +121,7 @@ struct DecodeParams {
 
 struct Bars {
   uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_conv[kStages];   // FP8 cache: the stage has been widened to bf16 (4 sender warps)
   uint64_t q_full, q_empty;
   uint64_t s_full;       // QK product of the current page is in S
   uint64_t s_read;       // the sender has read S (the next QK may overwrite it)
@@ -182,9 +203,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// kFp8: the cache pool holds FP8 rows (tm_kv = the codes as bytes, tm_scale =
+// the scales as bytes, tm_rope = the bf16 RoPE columns); otherwise bf16 rows
+// (tm_kv = the latent columns, tm_rope = the RoPE columns, tm_scale unused).
+template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rope,
-                  const DecodeParams p) {
+                  const __grid_constant__ CUtensorMap tm_scale, const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_kv = smem + kOffKV;
@@ -213,6 +238,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
+      if (kFp8) mbar_init(&bars->kv_conv[s], 4);
     }
     mbar_init(&bars->q_full, 4);       // the 4 q_lat / q_rope loader warps
     mbar_init(&bars->q_empty, 1);
@@ -241,6 +267,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     fence_mbar_init();
     prefetch_tmap(&tm_kv);
     prefetch_tmap(&tm_rope);
+    if (kFp8) prefetch_tmap(&tm_scale);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -307,11 +334,22 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             }
             uint8_t* st = s_kv + s * kStageBytes;
             const int y = pg + 1 == pe ? -shift : 0;   // first row of the block to load
-            mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);   // zero-filled bytes count too
+            if constexpr (kFp8) {
+              mbar_arrive_expect_tx(&bars->kv_full[s], kF8StageTx);
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tma_load_3d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, y, blk);
-            tma_load_3d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, y, blk);
+              for (int h = 0; h < 2; ++h)
+                tma_load_3d(st + (2 * h + 1) * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 128 * h, y, blk);
+#pragma unroll
+              for (int w4 = 0; w4 < kPage / kF8ScaleKeys; ++w4)
+                tma_load_3d(st + 2048 * w4, &tm_scale, &bars->kv_full[s], 0, y + kF8ScaleKeys * w4, blk);
+              tma_load_3d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 32 * rank, y, blk);
+            } else {
+              mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);   // zero-filled bytes count too
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                tma_load_3d(st + c * kChunkBytes, &tm_kv, &bars->kv_full[s], 256 * rank + 64 * c, y, blk);
+              tma_load_3d(st + 4 * kChunkBytes, &tm_rope, &bars->kv_full[s], 512 + 32 * rank, y, blk);
+            }
           }
         }
         fail = __shfl_sync(0xffffffffu, fail, 0);
@@ -334,7 +372,8 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // both from TMEM.  S is single-buffered; the sender frees it (s_read) as
     // soon as it has copied the product out.  The whole warp runs the loop
     // (descriptors stay warp-uniform) and one elected lane issues.
-    const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);
+    const uint32_t idesc_qk = idesc_bf16(128, 64, 0, 0);                                // RoPE half
+    const uint32_t idesc_lat = kFp8 ? idesc_f16(128, 64, 0, 0) : idesc_qk;              // latent half
     const uint64_t kv_desc0 = sdesc(smem_u32(s_kv), 16, 1024, kSwizzle128B);
     const uint64_t kr_desc0 = sdesc(smem_u32(s_kv) + 4 * kChunkBytes, 16, 512, kSwizzle64B);
     const uint64_t qr_desc = sdesc(smem_u32(s_qrope), 16, 512, kSwizzle64B);
@@ -347,6 +386,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       for (int j = 0; j < n; ++j, ++g) {
         const int s = g % kStages;
         if (!warp_wait(&bars->kv_full[s], (g / kStages) & 1, wc) ||
+            (kFp8 && !warp_wait(&bars->kv_conv[s], (g / kStages) & 1, wc)) ||
             (g > 0 && !warp_wait(&bars->s_read, (g - 1) & 1, wc))) {
           ok = false;
           break;
@@ -357,7 +397,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 #pragma unroll
         for (int t = 0; t < 16; ++t)   // latent half: K = 256 in steps of 16, A = q_lat from TMEM
           mma_ts_elect(tmem + kTmemS, tmem + kTmemQ + 8 * t,
-                       kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_qk, t != 0);
+                       kvd + (uint64_t)(((t >> 2) * kChunkBytes + (t & 3) * 32) >> 4), idesc_lat, t != 0);
 #pragma unroll
         for (int t = 0; t < 2; ++t)    // RoPE half: K = 32, A = q_rope from shared memory
           mma_ss_elect(tmem + kTmemS, qr_desc + (uint64_t)(t * 2), krd + (uint64_t)(t * 2), idesc_qk, 1);
@@ -377,7 +417,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // O += P . c_KV: M = 128 rows, N = 256 latent columns, K = 64 keys in 4
     // MMAs, A = P (bf16 pairs) from TMEM buffer g & 1, B = the stage's c_KV
     // half (MN-major).  Warp-wide loop, one elected lane issues.
-    const uint32_t idesc_pv = idesc_bf16(128, 256, 0, 1);
+    const uint32_t idesc_pv = kFp8 ? idesc_f16(128, 256, 0, 1) : idesc_bf16(128, 256, 0, 1);
     const uint64_t v_desc0 = sdesc(smem_u32(s_kv), kChunkBytes, 1024, kSwizzle128B);
     bool ok = true;
     int g = 0;
@@ -426,7 +466,58 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
+    // FP8 cache: widen stage gg to fp16 in place.  Thread = (key cr, code
+    // block ch).  Its 128 codes sit in chunk 2ch + 1, row cr; it writes the
+    // block's 128 fp16 columns to chunks 2ch (codes 0-63) and 2ch + 1 (codes
+    // 64-127, over its own codes, all read by then), so no thread overwrites
+    // bytes another thread still reads, except the scales in chunk 0: read
+    // first, then the warp syncs.  Page g + 2 is widened right after page g's
+    // scores have gone out: neither the score exchange nor the next QK
+    // product waits for it.
+    auto widen = [&](int gg) -> bool {
+      const int s = gg % kStages;
+      if (!warp_wait(&bars->kv_full[s], (gg / kStages) & 1, wc)) return false;
+      const int w4 = warp - 3, ch = lane >> 4;
+      // (recomputed per call: kept live across the sender loop they cost registers)
+      int cr;
+      asm volatile("mov.b32 %0, %1;" : "=r"(cr) : "r"(kF8ScaleKeys * w4 + (lane & 15)));
+      const uint32_t st = smem_u32(s_kv + s * kStageBytes);
+      const uint32_t s2 = pack_f16(ld_shared_f32(st + 2048 * w4 + (lane & 15) * 16 + (2 * rank + ch) * 4), 0.f);
+      __syncwarp();   // lanes 0 and 1 overwrite the warp's scales below
+      const uint32_t sc2 = __byte_perm(s2, 0, 0x1010);   // (s, s) in fp16
+      const uint32_t row = st + 2 * ch * kChunkBytes + cr * 128;
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {   // codes [64 hb, 64 hb + 64) -> fp16 chunk 2ch + hb
+        uint4 raw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) raw[k] = ld_shared_v4(row + kChunkBytes + (((4 * hb + k) ^ (cr & 7)) << 4));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // 16 codes -> fp16 16-byte chunks 2k, 2k + 1
+          const uint32_t wd[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            o[2 * i] = dequant_e4m3x2_f16(wd[i], sc2);
+            o[2 * i + 1] = dequant_e4m3x2_f16(wd[i] >> 16, sc2);
+          }
+          const uint32_t a = row + hb * kChunkBytes;
+          st_shared_v4(a + (((2 * k) ^ (cr & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
+          st_shared_v4(a + (((2 * k + 1) ^ (cr & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
+        }
+      }
+      fence_proxy_async_smem();   // read by the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->kv_conv[s]);
+      return true;
+    };
     int g = 0;
+    int pages_total = 0;   // pages of this cluster's items (FP8 cache: the widening runs two pages ahead)
+    if constexpr (kFp8) {
+      for (int it = it_begin; it < it_end; ++it)
+        pages_total += items[(size_t)it * kItemWords + kItPageEnd] - items[(size_t)it * kItemWords + kItPageBegin];
+      for (int gg = 0; gg < 2 && gg < pages_total; ++gg)
+        if (!widen(gg)) goto sender_fail;
+    }
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
       const int ii = it - it_begin;
@@ -447,16 +538,30 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         }
         const uint4* src = reinterpret_cast<const uint4*>(p.q_lat + ((size_t)w[kItRow] * p.n_heads + r) * 512 +
                                                           256 * rank);
+        if constexpr (kFp8) {   // the latent products take fp16 operands: 32 columns at a time
+#pragma unroll 1
+          for (int hq = 0; hq < 4; ++hq) {
+            uint32_t v[32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t v[64];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const uint4 q = r < p.n_heads ? __ldg(src + 16 * hh + k) : make_uint4(0, 0, 0, 0);
-            v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
+            for (int k = 0; k < 8; ++k) {
+              const uint4 q = r < p.n_heads ? __ldg(src + 8 * hq + k) : make_uint4(0, 0, 0, 0);
+              v[4 * k] = bf16x2_to_f16x2(q.x); v[4 * k + 1] = bf16x2_to_f16x2(q.y);
+              v[4 * k + 2] = bf16x2_to_f16x2(q.z); v[4 * k + 3] = bf16x2_to_f16x2(q.w);
+            }
+            tmem_st32(tmem + lane_addr + kTmemQ + 32 * hq, v);
           }
-          tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        } else {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t v[64];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const uint4 q = r < p.n_heads ? __ldg(src + 16 * hh + k) : make_uint4(0, 0, 0, 0);
+              v[4 * k] = q.x; v[4 * k + 1] = q.y; v[4 * k + 2] = q.z; v[4 * k + 3] = q.w;
+            }
+            tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(v));
+            tmem_st32(tmem + lane_addr + kTmemQ + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -490,6 +595,9 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         fence_proxy_async_smem();   // the copy warp's bulk copy reads the tile through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->own_full);
+        if constexpr (kFp8) {
+          if (g + 2 < pages_total && !widen(g + 2)) goto sender_fail;
+        }
       }
     }
     goto sender_done;
@@ -670,7 +778,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           float x0, x1;
           add_f16x2_to_f32(s2[k], nb, x0, x1);   // exact score + nb, rounded once
           const float e0 = ex2(x0), e1 = ex2(x1);
-          pk[k] = pack_bf16(e0, e1);
+          pk[k] = kFp8 ? pack_f16(e0, e1) : pack_bf16(e0, e1);
           ps[k & 3] += e0 + e1;
         }
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
@@ -799,30 +907,50 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
 
 // Set once per process, so that later launches can be captured in a CUDA graph.
+template <bool kFp8>
 cudaError_t decode_smem_attr() {
   static cudaError_t e =
-      cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      cudaFuncSetAttribute(mla_decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   return e;
 }
 
-}  // namespace
-
-mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+template <bool kFp8>
+mla_status_t launch_decode_impl(const mla_dims_t& d, const void* q_lat, const void* q_rope,
                                 const void* kv_pool, const int32_t* block_table,
                                 const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream) {
   // The pool as (column, row within the block, block): a box may start at a
   // negative row, which the TMA fills with zeros (the shifted last page).
-  CUtensorMap tm_kv, tm_rope;
-  const uint64_t pdims[3] = {576, (uint64_t)kPage, (uint64_t)d.num_blocks};
-  const uint64_t pstr[2] = {576 * 2, (uint64_t)kPage * 576 * 2};
-  const uint32_t box_kv[3] = {64, kPage, 1};
-  const uint32_t box_rope[3] = {32, kPage, 1};
-  mla_status_t st = encode_tmap_bf16(&tm_kv, kv_pool, 3, pdims, pstr, box_kv, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st != MLA_OK) return st;
-  st = encode_tmap_bf16(&tm_rope, kv_pool, 3, pdims, pstr, box_rope, CU_TENSOR_MAP_SWIZZLE_64B);
-  if (st != MLA_OK) return st;
+  CUtensorMap tm_kv, tm_rope, tm_scale;
+  mla_status_t st;
+  if constexpr (kFp8) {
+    const uint64_t rstr[2] = {kF8Row, (uint64_t)kPage * kF8Row};
+    const uint64_t cdims[3] = {512, (uint64_t)kPage, (uint64_t)d.num_blocks};
+    const uint32_t box_c[3] = {128, kPage, 1};
+    st = encode_tmap_u8(&tm_kv, kv_pool, 3, cdims, rstr, box_c, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != MLA_OK) return st;
+    const uint64_t sdims[3] = {16, (uint64_t)kPage, (uint64_t)d.num_blocks};
+    const uint32_t box_s[3] = {16, kF8ScaleKeys, 1};
+    st = encode_tmap_u8(&tm_scale, static_cast<const uint8_t*>(kv_pool) + kF8ScaleOff, 3, sdims, rstr, box_s,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != MLA_OK) return st;
+    const uint64_t rdims[3] = {64, (uint64_t)kPage, (uint64_t)d.num_blocks};
+    const uint32_t box_r[3] = {32, kPage, 1};
+    st = encode_tmap_bf16(&tm_rope, static_cast<const uint8_t*>(kv_pool) + kF8RopeOff, 3, rdims, rstr, box_r,
+                          CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != MLA_OK) return st;
+  } else {
+    const uint64_t pdims[3] = {576, (uint64_t)kPage, (uint64_t)d.num_blocks};
+    const uint64_t pstr[2] = {576 * 2, (uint64_t)kPage * 576 * 2};
+    const uint32_t box_kv[3] = {64, kPage, 1};
+    const uint32_t box_rope[3] = {32, kPage, 1};
+    st = encode_tmap_bf16(&tm_kv, kv_pool, 3, pdims, pstr, box_kv, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != MLA_OK) return st;
+    st = encode_tmap_bf16(&tm_rope, kv_pool, 3, pdims, pstr, box_rope, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != MLA_OK) return st;
+    tm_scale = tm_rope;   // unused
+  }
   const int N = d.B * d.s_q;
 
   DecodeParams p;
@@ -848,13 +976,34 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
 
-  cudaError_t e = decode_smem_attr();
+  cudaError_t e = decode_smem_attr<kFp8>();
   if (e == cudaSuccess) {
-    e = launch_pdl(mla_decode_kernel, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv, tm_rope, p);
+    e = launch_pdl(mla_decode_kernel<kFp8>, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv,
+                   tm_rope, tm_scale, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   return MLA_OK;
+}
+
+}  // namespace
+
+mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+                                const void* kv_pool, const int32_t* block_table,
+                                const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
+                                int32_t num_clusters, float* o_part, float* lse_part,
+                                void* o_lat, float* lse_out, int32_t* status, void* stream) {
+  return launch_decode_impl<false>(d, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_masks, plan_dev,
+                                   num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
+}
+
+mla_status_t launch_decode_attn_fp8cache(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+                                         const void* kv_pool_fp8, const int32_t* block_table,
+                                         const int32_t* seq_lens, const int32_t* plan_dev, int32_t num_clusters,
+                                         float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                                         int32_t* status, void* stream) {
+  return launch_decode_impl<true>(d, q_lat, q_rope, kv_pool_fp8, block_table, seq_lens, nullptr, plan_dev,
+                                  num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
 }
 
 void set_decode_wait_limit_ns(int64_t ns) {
@@ -862,7 +1011,7 @@ void set_decode_wait_limit_ns(int64_t ns) {
 }
 
 mla_status_t decode_max_clusters(int32_t* n) {
-  cudaError_t e = decode_smem_attr();
+  cudaError_t e = decode_smem_attr<false>();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "max clusters: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
@@ -876,7 +1025,7 @@ mla_status_t decode_max_clusters(int32_t* n) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int count = 0;
-  e = cudaOccupancyMaxActiveClusters(&count, mla_decode_kernel, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&count, mla_decode_kernel<false>, &cfg);
   if (e != cudaSuccess || count <= 0) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);

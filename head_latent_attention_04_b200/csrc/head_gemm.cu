@@ -395,6 +395,40 @@ __global__ void quantize_rows_kernel(const __nv_bfloat16* __restrict__ x, long l
   }
 }
 
+// New cache rows -> FP8 latent-cache slots (row = 512 E4M3 codes | 4 fp32
+// scales | 64 bf16 k_rope, 656 bytes).  Thread = (row, 128-column block): the
+// same quantiser as the activations, plus a quarter of the row's k_rope.
+constexpr int kKvRow = 576, kF8CacheRow = 656;
+
+__global__ void kv_quantize_fp8_kernel(const __nv_bfloat16* __restrict__ kv, const int32_t* __restrict__ slots,
+                                       long long n, uint8_t* __restrict__ pool, long long pool_rows,
+                                       int32_t* status) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < 4 * n; i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i >> 2;
+    const int j = (int)(i & 3);
+    const long long slot = slots[row];
+    if (slot < 0 || slot >= pool_rows) {
+      if (status && j == 0) atomicOr(status, MLA_STATUS_BAD_BLOCK);
+      continue;
+    }
+    const __nv_bfloat16* src = kv + row * kKvRow;
+    uint8_t* dst = pool + slot * kF8CacheRow;
+    uint4 v[16];
+    load128(src + 128 * j, v);
+    uint32_t q[32];
+    const float s = quant128(v, q);
+    if (status && s > 65504.f / kE4M3Max) atomicOr(status, MLA_STATUS_CACHE_RANGE);   // widened in fp16
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      reinterpret_cast<uint4*>(dst + 128 * j)[c] = make_uint4(q[4 * c], q[4 * c + 1], q[4 * c + 2], q[4 * c + 3]);
+    reinterpret_cast<float*>(dst + 512)[j] = s;
+    const uint4* rs = reinterpret_cast<const uint4*>(src + 512) + 2 * j;   // k_rope bytes [32j, 32j + 32)
+    uint4* rd = reinterpret_cast<uint4*>(dst + 528) + 2 * j;
+    rd[0] = __ldg(rs);
+    rd[1] = __ldg(rs + 1);
+  }
+}
+
 // absorb, FP8: one CTA per (128-row tile of the head's W_UK codes, head, token
 // tile).  A = codes [128 k][128 d] (one TMA box, SW128); the tokens' q_nope rows
 // arrive by TMA as bf16 (two SW128 chunks of 64 d, as in the bf16 kernel) and
@@ -744,6 +778,17 @@ mla_status_t launch_quantize_rows_fp8(const void* x, long long rows, int cols, v
       static_cast<const __nv_bfloat16*>(x), n_vec, static_cast<uint8_t*>(codes), scales);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "quantize_rows launch: %s", cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+mla_status_t launch_kv_quantize_fp8(const void* kv, const int32_t* slots, long long n, void* pool_fp8,
+                                   long long pool_rows, int32_t* status, void* stream) {
+  if (n == 0) return MLA_OK;
+  const long long blocks = (4 * n + 127) / 128;
+  kv_quantize_fp8_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(kv), slots, n, static_cast<uint8_t*>(pool_fp8), pool_rows, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "kv_quantize_fp8 launch: %s", cudaGetErrorString(e));
   return MLA_OK;
 }
 

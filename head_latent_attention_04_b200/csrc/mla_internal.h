@@ -54,6 +54,16 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
                                 const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream);
+// The same kernel on an FP8 latent cache (rows of 656 bytes: 512 E4M3 codes,
+// 4 fp32 block scales, 64 bf16 k_rope).  No draft-tree masks.
+mla_status_t launch_decode_attn_fp8cache(const mla_dims_t& d, const void* q_lat, const void* q_rope,
+                                         const void* kv_pool_fp8, const int32_t* block_table,
+                                         const int32_t* seq_lens, const int32_t* plan_dev, int32_t num_clusters,
+                                         float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                                         int32_t* status, void* stream);
+// bf16 cache rows [n][576] -> FP8 pool slots (flat token index block * 64 + row).
+mla_status_t launch_kv_quantize_fp8(const void* kv, const int32_t* slots, long long n, void* pool_fp8,
+                                   long long pool_rows, int32_t* status, void* stream);
 mla_status_t launch_combine(const mla_dims_t& d, const int32_t* plan_dev, int32_t n_rows,
                             const float* o_part, const float* lse_part, void* o_lat,
                             float* lse_out, void* stream);

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -209,6 +210,19 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
 }
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+// 16-byte and 4-byte shared-memory loads at a shared::cta address.
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 // 16-byte shared-memory store at a shared::cta address.
@@ -478,6 +492,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          ((uint32_t)(N >> 3) << 17)         // N / 8
          | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
+// The same with fp16 A/B (format code 0).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn) {
+  return idesc_bf16(M, N, a_mn, b_mn) & ~((1u << 7) | (1u << 10));
+}
 
 // Instruction descriptor for kind::f8f6f4 with E4M3 A and B (format code 0),
 // both K-major, and fp32 D.
@@ -515,6 +533,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;   // low 16 bits = lo, high 16 bits = hi, each rounded to nearest even
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// Two E4M3 codes (low byte first) times a block scale -> fp16 pair: each code
+// is widened exactly (E4M3 values are fp16 values), then multiplied by the
+// scale pair s2 = (s, s) in fp16, rounded once.
+__device__ __forceinline__ uint32_t dequant_e4m3x2_f16(uint32_t codes16, uint32_t s2) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes16 & 0xFFFFu), __NV_E4M3);
+  const uint32_t x = (uint32_t)h.x | ((uint32_t)h.y << 16);
+  uint32_t y;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(y) : "r"(x), "r"(s2));
+  return y;
+}
+
+// bf16 pair -> fp16 pair (each value widened exactly, then rounded once).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t u) {
+  return pack_f16(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 
 }  // namespace ptx

@@ -24,12 +24,14 @@ _lib = ctypes.CDLL(_LIB_PATH)
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED = 0, 1, 2
 MLA_ERR_WORKSPACE_TOO_SMALL, MLA_ERR_CUDA, MLA_ERR_TIMEOUT = 3, 4, 5
 STATUS_BAD_BLOCK, STATUS_TIMEOUT, STATUS_BAD_SEQLEN, STATUS_BAD_PLAN, STATUS_SCORE_RANGE = 0x1, 0x2, 0x4, 0x8, 0x10
+STATUS_CACHE_RANGE = 0x20
 EXPORTS = ("mla_version", "mla_last_error_string", "mla_absorb_q", "mla_out_uv",
            "mla_max_clusters", "mla_plan_size", "mla_plan", "mla_decode_attn", "mla_combine",
            "mla_debug_gather_pages", "mla_decode_attn_combine_noalloc", "mla_noalloc_scratch_bytes",
            "mla_quantize_w_uk_fp8", "mla_quantize_w_uv_fp8", "mla_quantize_rows_fp8", "mla_absorb_q_fp8",
            "mla_out_uv_fp8", "mla_set_wait_limit_ns", "mla_decode_attn_tree", "mla_prefill_up_proj",
-           "mla_prefill_attn", "mla_qkv_a_proj", "mla_q_up_absorb")
+           "mla_prefill_attn", "mla_qkv_a_proj", "mla_q_up_absorb", "mla_decode_attn_fp8cache",
+           "mla_kv_quantize_fp8")
 
 
 class MlaDims(ctypes.Structure):
@@ -52,6 +54,8 @@ for _name, _args in {
     "mla_plan": [_pdims, _vp, _i32, _vp, _sz, ctypes.POINTER(_i32)],
     "mla_decode_attn": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_decode_attn_tree": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
+    "mla_decode_attn_fp8cache": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
+    "mla_kv_quantize_fp8": [_vp, _vp, ctypes.c_int64, _vp, _i32, _vp, _vp],
     "mla_combine": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp],
     "mla_debug_gather_pages": [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp],
     "mla_decode_attn_combine_noalloc": [_pdims, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _i32, _vp, _vp, _vp, _vp],
@@ -240,6 +244,36 @@ def decode_attn_tree(dims, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_
                                      _ptr(status), _stream(stream)), "mla_decode_attn_tree")
 
 
+FP8_ROW_BYTES = 656   # 512 E4M3 codes | 4 fp32 block scales | 64 bf16 k_rope
+
+
+def decode_attn_fp8cache(dims, q_lat, q_rope, kv_pool_fp8, block_table, seq_lens, plan_dev, num_clusters,
+                         o_part, lse_part, o_lat, lse_out=None, status=None, stream=None):
+    """decode_attn on an FP8 latent cache: ``kv_pool_fp8`` uint8
+    [num_blocks][64][656] as :func:`kv_quantize_fp8` writes it."""
+    _check(_lib.mla_decode_attn_fp8cache(ctypes.byref(dims), _ptr(q_lat), _ptr(q_rope), _ptr(kv_pool_fp8),
+                                         _ptr(block_table), _ptr(seq_lens), _ptr(plan_dev), num_clusters,
+                                         _ptr(o_part), _ptr(lse_part), _ptr(o_lat), _ptr(lse_out),
+                                         _ptr(status), _stream(stream)), "mla_decode_attn_fp8cache")
+
+
+def kv_quantize_fp8(kv, slots, kv_pool_fp8, status=None, stream=None):
+    """bf16 cache rows ``kv`` [n][576] -> slots ``slots`` (int32 [n], block * 64 +
+    row) of the FP8 pool (uint8 [num_blocks][64][656])."""
+    n = kv.numel() // 576
+    _check(_lib.mla_kv_quantize_fp8(_ptr(kv), _ptr(slots), n, _ptr(kv_pool_fp8), kv_pool_fp8.shape[0],
+                                    _ptr(status), _stream(stream)), "mla_kv_quantize_fp8")
+    return kv_pool_fp8
+
+
+def fp8_pool_from(kv_pool, stream=None):
+    """The FP8 copy of a whole bf16 pool [num_blocks][64][576] (every slot quantised)."""
+    nb = kv_pool.shape[0]
+    pool8 = torch.empty((nb, 64, FP8_ROW_BYTES), dtype=torch.uint8, device=kv_pool.device)
+    slots = torch.arange(nb * 64, dtype=torch.int32, device=kv_pool.device)
+    return kv_quantize_fp8(kv_pool.reshape(nb * 64, 576), slots, pool8, stream=stream)
+
+
 def combine(dims, plan_dev, o_part, lse_part, o_lat, lse_out=None, stream=None):
     _check(_lib.mla_combine(ctypes.byref(dims), _ptr(plan_dev), _ptr(o_part), _ptr(lse_part),
                             _ptr(o_lat), _ptr(lse_out), _stream(stream)), "mla_combine")
@@ -344,7 +378,13 @@ class Decoder:
     """
 
     def __init__(self, seq_lens, s_q: int, n_heads: int, max_blocks: int, num_blocks: int,
-                 device="cuda", scale=None, causal=True, num_clusters: int | None = None):
+                 device="cuda", scale=None, causal=True, num_clusters: int | None = None,
+                 kv_cache: str = "bf16"):
+        """``kv_cache``: "bf16" (pool [num_blocks][64][576] bf16) or "fp8" (pool
+        uint8 [num_blocks][64][656], see :func:`kv_quantize_fp8`)."""
+        if kv_cache not in ("bf16", "fp8"):
+            raise ValueError("kv_cache must be 'bf16' or 'fp8'")
+        self.kv_cache = kv_cache
         self.seq_lens_host = np.asarray(seq_lens, dtype=np.int32)
         self.B = len(self.seq_lens_host)
         self.s_q, self.H = s_q, n_heads
@@ -381,7 +421,13 @@ class Decoder:
             absorb_q_fp8(q_nope, self.fp8_uk, self.q_lat, stream)
         else:
             absorb_q(q_nope, w_uk, self.q_lat, stream)
-        if draft_masks is not None:
+        if draft_masks is not None and self.kv_cache == "fp8":
+            raise ValueError("draft-tree masks need the bf16 cache")
+        if self.kv_cache == "fp8":
+            decode_attn_fp8cache(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev,
+                                 self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
+                                 self.lse, self.status, stream)
+        elif draft_masks is not None:
             decode_attn_tree(self.dims, self.q_lat, q_rope, kv_pool, block_table, self.seq_lens_dev, draft_masks,
                              self.plan_dev, self.num_clusters, self.o_part, self.lse_part, self.o_lat,
                              self.lse, self.status, stream)

@@ -63,6 +63,9 @@ typedef enum {
                                         nothing computed */
 #define MLA_STATUS_SCORE_RANGE 0x10  /* a partial score of an attended key left the fp16 range
                                         (|x| > 65504) or was not a number: outputs are invalid */
+#define MLA_STATUS_CACHE_RANGE 0x20  /* mla_kv_quantize_fp8: a 128-column block of c_KV has
+                                        amax > 65504, beyond what mla_decode_attn_fp8cache widens
+                                        (fp16); the row is written but must not be attended */
 
 /* Problem dimensions of one decode batch. */
 typedef struct {
@@ -232,6 +235,48 @@ mla_status_t mla_decode_attn_tree(const mla_dims_t* dims, const void* q_lat, con
                                   const int32_t* draft_masks, const void* plan_dev, int32_t num_clusters,
                                   float* o_part, float* lse_part, void* o_lat, float* lse_out,
                                   int32_t* status, void* stream);
+
+/*
+ * mla_decode_attn_fp8cache -- mla_decode_attn on an FP8 latent cache.  The
+ * pages quantise activations in 128-element blocks with one scale each ("Lower
+ * latency and higher throughput with multi-node DeepSeek deployment", section
+ * "Quantization"); applied to the cached c_KV row that halves the bytes the
+ * decode streams per token (656 instead of 1152), the cache-size argument of
+ * the izhida.com answer.  Token row layout (656 bytes, 16-byte multiple):
+ *   bytes [0, 512)    E4M3 codes of c_KV[t, 0..511]
+ *   bytes [512, 528)  fp32 scales s_0..s_3, c_KV[t, c] = code[c] * s_{c / 128}
+ *   bytes [528, 656)  k_rope[t, 0..63] in bf16 (not quantised)
+ *   kv_pool_fp8  uint8 [num_blocks][64][656], 16-byte aligned (mla_kv_quantize_fp8 writes it)
+ * Numerics: the kernel widens every staged row to fp16 (code * fp16(scale),
+ * rounded once), rounds q_lat to fp16 and writes P as fp16, and runs the
+ * latent products on those fp16 operands (fp32 accumulation); the RoPE
+ * products are bf16 as in mla_decode_attn.  Blocks need amax <= 65504 (see
+ * MLA_STATUS_CACHE_RANGE) and q_lat |x| <= 65504 (beyond, the scores become
+ * infinite and MLA_STATUS_SCORE_RANGE is set).  All other arguments, outputs,
+ * status bits and the plan are those of mla_decode_attn; mla_combine
+ * completes split rows.  No draft-tree masks.
+ */
+mla_status_t mla_decode_attn_fp8cache(const mla_dims_t* dims, const void* q_lat, const void* q_rope,
+                                      const void* kv_pool_fp8, const int32_t* block_table,
+                                      const int32_t* seq_lens, const void* plan_dev, int32_t num_clusters,
+                                      float* o_part, float* lse_part, void* o_lat, float* lse_out,
+                                      int32_t* status, void* stream);
+
+/*
+ * mla_kv_quantize_fp8 -- write cache rows into FP8 pool slots (the layout of
+ * mla_decode_attn_fp8cache).  Per 128-column block of c_KV: amax = max |x|,
+ * s = amax / 448, code = E4M3(x * (448 / amax)) rounded to nearest even and
+ * saturated (an all-zero block takes s = 1); k_rope is copied.
+ *   kv        bf16 [n][576]  rows c_KV (512) | k_rope (64), 16-byte aligned
+ *   slots     int32 [n]      destination of row i: block * 64 + row in the block
+ *   pool_fp8  uint8 [num_blocks][64][656]
+ *   status    int32 [1] or NULL: MLA_STATUS_BAD_BLOCK when a slot lies outside
+ *             the pool (that row is not written); MLA_STATUS_CACHE_RANGE when a
+ *             block's amax exceeds 65504 (written, but not attendable)
+ * Rows with equal slots race (one of them wins).
+ */
+mla_status_t mla_kv_quantize_fp8(const void* kv, const int32_t* slots, int64_t n, void* pool_fp8,
+                                 int32_t num_blocks, int32_t* status, void* stream);
 
 /*
  * mla_combine -- log-sum-exp merge of the split pieces of each split row:
