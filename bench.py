@@ -66,6 +66,11 @@ def parse_args(argv=None):
                     help="latent cache rows as bf16 (1152 B/token) or E4M3 codes with fp32 block scales "
                          "and a bf16 k_rope (656 B/token)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--path", default="decode", choices=["decode", "prefill", "upstream"],
+                    help="decode: the absorbed decode step (the headline line); prefill: order-1 prefill of one "
+                         "sequence (--prefill T,s); upstream: qkv_a_proj and q_up_absorb for --tokens rows")
+    ap.add_argument("--prefill", default="4096,4096", help="T,s of the prefill path (s = T: full prefill)")
+    ap.add_argument("--tokens", type=int, default=256, help="token rows of the upstream path")
     return ap.parse_args(argv)
 
 
@@ -509,8 +514,106 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     return res
 
 
+# ----------------------------------------------------------------------------- the NEXT paths
+def _time_kernel(fn, K, W, flush, stream):
+    """Mean CUDA-event time (ms) of fn() over K runs after W warm-ups, L2 flushed before each."""
+    import torch
+    for _ in range(max(W, 3)):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.fmean(a.elapsed_time(b) for a, b in ev)
+
+
+def _roof(flops, nbytes, ms, peaks, peak_src):
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    src = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'}, burst)"
+    if t_tensor > t_hbm:
+        a = flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": a / peaks["bf16_tflops"], "alg_flops": flops, "alg_bytes": nbytes, "kernel_ms": ms,
+                "peak_source": src}
+    a = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": a / peaks["hbm_gbs"],
+            "alg_flops": flops, "alg_bytes": nbytes, "kernel_ms": ms, "peak_source": src}
+
+
+def run_next_path(args):
+    """One JSON line for the prefill or upstream path (one GPU): each kernel timed
+    with CUDA events on its own, L2 flushed before every run, with its roofline."""
+    import torch
+    from head_latent_attention_04_b200 import mla
+    from head_latent_attention_04_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    peaks, peak_src = load_peaks()
+    K, Wm = args.steps, args.warmup
+    H = 128
+    if args.path == "prefill":
+        T, s = (int(x) for x in args.prefill.split(","))
+        w = W.make_workload(1, s, H, [T], seed=7, pool="permuted", device=dev)
+        row = torch.as_tensor(w.block_table[0], dtype=torch.int32, device=dev)
+        k = torch.empty((T, H, 128), dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+        out = torch.empty((s, H, 128), dtype=torch.bfloat16, device=dev)
+        up = lambda: mla.prefill_up_proj(w.kv_pool, row, T, w.w_uk, w.w_uv, k, v)
+        attn = lambda: mla.prefill_attn(w.q_nope, w.q_rope, k, v, w.kv_pool, row, T, out=out)
+        ms_up = _time_kernel(up, K, Wm, flush, stream)
+        ms_attn = _time_kernel(attn, K, Wm, flush, stream)
+        pairs = sum(T - s + 1 + i for i in range(s))
+        kern = {
+            "up_proj_kernel": _roof(2 * 2 * T * 512 * 128 * H, T * 1152 + 2 * 512 * H * 128 * 2 + 2 * T * H * 128 * 2,
+                                    ms_up, peaks, peak_src),
+            "prefill_attn_kernel": _roof(pairs * H * 2 * (192 + 128),
+                                         s * H * (192 + 128) * 2 + 2 * T * H * 128 * 2 + T * 128 + s * H * 4,
+                                         ms_attn, peaks, peak_src),
+        }
+        ms = ms_up + ms_attn
+        tokens, workload = s, {"workload": f"prefill T={T} s={s}", "n_heads": H, "pool": "permuted", "seed": 7}
+    else:
+        N = args.tokens
+        g = torch.Generator(device=dev)
+        g.manual_seed(9)
+        rnd = lambda shape, std: (torch.randn(shape, generator=g, device=dev) * std).to(torch.bfloat16)
+        x = rnd((N, 7168), 1.0)
+        w_qkv = rnd((2112, 7168), 7168 ** -0.5)
+        c_q = rnd((N, 1536), 1.0)
+        w_uq = rnd((1536, H, 192), 1536 ** -0.5)
+        w_uk = rnd((512, H, 128), 512 ** -0.5)
+        ms_a = _time_kernel(lambda: mla.qkv_a_proj(x, w_qkv), K, Wm, flush, stream)
+        ms_b = _time_kernel(lambda: mla.q_up_absorb(c_q, w_uq, w_uk), K, Wm, flush, stream)
+        kern = {
+            "qkv_a_proj_kernel": _roof(2 * N * 7168 * 2112, 2112 * 7168 * 2 + N * 7168 * 2 + N * 2112 * 2,
+                                       ms_a, peaks, peak_src),
+            "q_up_absorb_kernel": _roof(2 * N * 1536 * H * 192 + 2 * N * H * 128 * 512,
+                                        1536 * H * 192 * 2 + 512 * H * 128 * 2 + N * 1536 * 2 + N * H * 576 * 2,
+                                        ms_b, peaks, peak_src),
+        }
+        ms = ms_a + ms_b
+        tokens, workload = N, {"workload": f"upstream N={N}", "n_heads": H, "seed": 9}
+    return {"metric": f"{args.path} tokens/s (kernels timed one by one)", "value": tokens / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic", "path": args.path,
+            "config": dict(workload, l2="flushed before every kernel run (256 MB write, outside the events)"),
+            "kernels": kern, "gpu_launches": 2 * K}
+
+
 def main(argv=None):
     args = parse_args(argv)
+    if args.path != "decode":
+        print(json.dumps(run_next_path(args)), flush=True)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -206,7 +206,10 @@ __device__ __forceinline__ float ex2(float x) {
 // kFp8: the cache pool holds FP8 rows (tm_kv = the codes as bytes, tm_scale =
 // the scales as bytes, tm_rope = the bf16 RoPE columns); otherwise bf16 rows
 // (tm_kv = the latent columns, tm_rope = the RoPE columns, tm_scale unused).
-template <bool kFp8>
+// kTree: p.draft_masks gives each query's view of the drafted tokens (an
+// instance of its own, so the other instances' softmax loop carries no mask
+// code: its instruction footprint was measured to cost 1-2 %).
+template <bool kFp8, bool kTree>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_rope,
                   const __grid_constant__ CUtensorMap tm_scale, const DecodeParams p) {
@@ -471,9 +474,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // block's 128 fp16 columns to chunks 2ch (codes 0-63) and 2ch + 1 (codes
     // 64-127, over its own codes, all read by then), so no thread overwrites
     // bytes another thread still reads, except the scales in chunk 0: read
-    // first, then the warp syncs.  Page g + 2 is widened right after page g's
-    // scores have gone out: neither the score exchange nor the next QK
-    // product waits for it.
+    // first, then the warp syncs.  Page g + 1 is widened before page g's
+    // scores are awaited (pages 0 and 1 before page 0's), that is, right after
+    // page g - 1's scores have gone out: neither the score exchange nor the
+    // next QK product waits for it.
     auto widen = [&](int gg) -> bool {
       const int s = gg % kStages;
       if (!warp_wait(&bars->kv_full[s], (gg / kStages) & 1, wc)) return false;
@@ -486,7 +490,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       __syncwarp();   // lanes 0 and 1 overwrite the warp's scales below
       const uint32_t sc2 = __byte_perm(s2, 0, 0x1010);   // (s, s) in fp16
       const uint32_t row = st + 2 * ch * kChunkBytes + cr * 128;
-#pragma unroll
+#pragma unroll 1
       for (int hb = 0; hb < 2; ++hb) {   // codes [64 hb, 64 hb + 64) -> fp16 chunk 2ch + hb
         uint4 raw[4];
 #pragma unroll
@@ -496,10 +500,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
           const uint32_t wd[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
           uint32_t o[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            o[2 * i] = dequant_e4m3x2_f16(wd[i], sc2);
-            o[2 * i + 1] = dequant_e4m3x2_f16(wd[i] >> 16, sc2);
-          }
+          for (int i = 0; i < 4; ++i) dequant_e4m3x4_f16(wd[i], sc2, o[2 * i], o[2 * i + 1]);
           const uint32_t a = row + hb * kChunkBytes;
           st_shared_v4(a + (((2 * k) ^ (cr & 7)) << 4), make_uint4(o[0], o[1], o[2], o[3]));
           st_shared_v4(a + (((2 * k + 1) ^ (cr & 7)) << 4), make_uint4(o[4], o[5], o[6], o[7]));
@@ -511,12 +512,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       return true;
     };
     int g = 0;
-    int pages_total = 0;   // pages of this cluster's items (FP8 cache: the widening runs two pages ahead)
+    int pages_total = 0, widened = 0;   // FP8 cache: this cluster's pages, and those widened so far
     if constexpr (kFp8) {
       for (int it = it_begin; it < it_end; ++it)
         pages_total += items[(size_t)it * kItemWords + kItPageEnd] - items[(size_t)it * kItemWords + kItPageBegin];
-      for (int gg = 0; gg < 2 && gg < pages_total; ++gg)
-        if (!widen(gg)) goto sender_fail;
     }
     for (int it = it_begin; it < it_end; ++it) {
       const int32_t* w = items + (size_t)it * kItemWords;
@@ -570,6 +569,10 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
       }
       const int n = w[kItPageEnd] - w[kItPageBegin];
       for (int j = 0; j < n; ++j, ++g) {
+        if constexpr (kFp8) {   // pages up to g + 1: at g = 0 pages 0 and 1, then one per page
+          for (; widened < min(g + 2, pages_total); ++widened)
+            if (!widen(widened)) goto sender_fail;
+        }
         uint32_t v[64];
         if (!warp_wait(&bars->s_full, g & 1, wc)) goto sender_fail;
         tc_fence_after();
@@ -595,9 +598,6 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
         fence_proxy_async_smem();   // the copy warp's bulk copy reads the tile through the async proxy
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->own_full);
-        if constexpr (kFp8) {
-          if (g + 2 < pages_total && !widen(g + 2)) goto sender_fail;
-        }
       }
     }
     goto sender_done;
@@ -653,7 +653,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
     // The sequence length of the next item is loaded one item ahead, so that
     // the stale-plan check never waits for memory at an item boundary.
     // So is the next item's draft mask, when drafts form a tree.
-    const bool tree = p.draft_masks != nullptr;
+    constexpr bool tree = kTree;
     int T_next = 0, m_next = 0;
     if (it_begin < it_end) {
       const int32_t* w0 = items + (size_t)it_begin * kItemWords;
@@ -731,7 +731,7 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
             if (32 * c + 2 * k + 1 < lo) s2[k] = (s2[k] & 0x0000ffffu) | 0xfc000000u;
           }
         }
-        if (tree) {
+        if constexpr (tree) {
           // draft keys: column col holds key (page start + col - shift); draft
           // d = key - first_draft is visible iff bit d of this row's mask is set
           const int col0 = first_draft - ((pb + j) * kPage - (j == n - 1 ? shift_last : 0));
@@ -907,14 +907,14 @@ mla_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_consta
 std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
 
 // Set once per process, so that later launches can be captured in a CUDA graph.
-template <bool kFp8>
+template <bool kFp8, bool kTree>
 cudaError_t decode_smem_attr() {
   static cudaError_t e =
-      cudaFuncSetAttribute(mla_decode_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      cudaFuncSetAttribute(mla_decode_kernel<kFp8, kTree>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   return e;
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kTree>
 mla_status_t launch_decode_impl(const mla_dims_t& d, const void* q_lat, const void* q_rope,
                                 const void* kv_pool, const int32_t* block_table,
                                 const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
@@ -976,9 +976,9 @@ mla_status_t launch_decode_impl(const mla_dims_t& d, const void* q_lat, const vo
   p.scale_log2 = d.scale * 1.4426950408889634f;
   p.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
 
-  cudaError_t e = decode_smem_attr<kFp8>();
+  cudaError_t e = decode_smem_attr<kFp8, kTree>();
   if (e == cudaSuccess) {
-    e = launch_pdl(mla_decode_kernel<kFp8>, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv,
+    e = launch_pdl(mla_decode_kernel<kFp8, kTree>, dim3(2 * num_clusters), dim3(kThreads), kSmemBytes, stream, tm_kv,
                    tm_rope, tm_scale, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
@@ -993,8 +993,11 @@ mla_status_t launch_decode_attn(const mla_dims_t& d, const void* q_lat, const vo
                                 const int32_t* seq_lens, const int32_t* draft_masks, const int32_t* plan_dev,
                                 int32_t num_clusters, float* o_part, float* lse_part,
                                 void* o_lat, float* lse_out, int32_t* status, void* stream) {
-  return launch_decode_impl<false>(d, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_masks, plan_dev,
-                                   num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
+  if (draft_masks)
+    return launch_decode_impl<false, true>(d, q_lat, q_rope, kv_pool, block_table, seq_lens, draft_masks, plan_dev,
+                                           num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
+  return launch_decode_impl<false, false>(d, q_lat, q_rope, kv_pool, block_table, seq_lens, nullptr, plan_dev,
+                                          num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
 }
 
 mla_status_t launch_decode_attn_fp8cache(const mla_dims_t& d, const void* q_lat, const void* q_rope,
@@ -1002,8 +1005,8 @@ mla_status_t launch_decode_attn_fp8cache(const mla_dims_t& d, const void* q_lat,
                                          const int32_t* seq_lens, const int32_t* plan_dev, int32_t num_clusters,
                                          float* o_part, float* lse_part, void* o_lat, float* lse_out,
                                          int32_t* status, void* stream) {
-  return launch_decode_impl<true>(d, q_lat, q_rope, kv_pool_fp8, block_table, seq_lens, nullptr, plan_dev,
-                                  num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
+  return launch_decode_impl<true, false>(d, q_lat, q_rope, kv_pool_fp8, block_table, seq_lens, nullptr, plan_dev,
+                                         num_clusters, o_part, lse_part, o_lat, lse_out, status, stream);
 }
 
 void set_decode_wait_limit_ns(int64_t ns) {
@@ -1011,7 +1014,7 @@ void set_decode_wait_limit_ns(int64_t ns) {
 }
 
 mla_status_t decode_max_clusters(int32_t* n) {
-  cudaError_t e = decode_smem_attr<false>();
+  cudaError_t e = decode_smem_attr<false, false>();
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "max clusters: %s", cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
@@ -1025,7 +1028,7 @@ mla_status_t decode_max_clusters(int32_t* n) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int count = 0;
-  e = cudaOccupancyMaxActiveClusters(&count, mla_decode_kernel<false>, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&count, mla_decode_kernel<false, false>, &cfg);
   if (e != cudaSuccess || count <= 0) {
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);

@@ -535,15 +535,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
-// Two E4M3 codes (low byte first) times a block scale -> fp16 pair: each code
-// is widened exactly (E4M3 values are fp16 values), then multiplied by the
-// scale pair s2 = (s, s) in fp16, rounded once.
-__device__ __forceinline__ uint32_t dequant_e4m3x2_f16(uint32_t codes16, uint32_t s2) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes16 & 0xFFFFu), __NV_E4M3);
-  const uint32_t x = (uint32_t)h.x | ((uint32_t)h.y << 16);
-  uint32_t y;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(y) : "r"(x), "r"(s2));
-  return y;
+// Four E4M3 codes (byte i = code i) times a block scale -> two fp16 pairs
+// (codes 0, 1 in lo; 2, 3 in hi): each code is widened exactly (E4M3 values
+// are fp16 values), then multiplied by the scale pair s2 = (s, s) in fp16,
+// rounded once.
+__device__ __forceinline__ void dequant_e4m3x4_f16(uint32_t codes, uint32_t s2, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 c01, c23;\n\t.reg .b32 x01, x23;\n\t"
+      "mov.b32 {c01, c23}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 x01, c01;\n\tcvt.rn.f16x2.e4m3x2 x23, c23;\n\t"
+      "mul.rn.f16x2 %0, x01, %3;\n\tmul.rn.f16x2 %1, x23, %3;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(codes), "r"(s2));
 }
 
 // bf16 pair -> fp16 pair (each value widened exactly, then rounded once).
