@@ -18,7 +18,8 @@
 //   tcgen05 GEMM, M = 128 features of the head's W_UK / W_UV slice, N = 128
 //   tokens (two cache pages, read through the block table by TMA from the
 //   (column, row, block) view of the pool), K = 512 latent columns streamed
-//   through a ring; the TMA-store epilogue writes K or V [T][h][128] bf16.
+//   through a three-stage ring (two CTAs per SM); the TMA-store epilogue
+//   writes K or V [T][h][128] bf16.
 // prefill_attn_kernel: one CTA per (128-query tile, head).  Warp 0 stages
 //   the Q tile once and K / k_rope / V tiles of 128 keys through a two-stage
 //   ring; warp 1 issues S = Q K^T (M = 128 queries, N = 128 keys, K = 192:
@@ -43,7 +44,7 @@ using namespace ptx;
 
 constexpr int kTile = 128;                 // tokens per tile (queries, keys, up-projection)
 constexpr int kChunk = kTile * 128;        // 16 KB: 128 rows x 64 bf16 (SW128)
-constexpr int kUpStages = 6;
+constexpr int kUpStages = 3;            // 97 KB: two CTAs per SM, so one's epilogue overlaps the other's loads
 constexpr int kUpStageBytes = 2 * kChunk;  // W chunk (two 64-feature halves) + c_KV chunk
 
 __device__ __forceinline__ void store_rows(uint32_t tmem, uint8_t* s_out, const CUtensorMap* tm_out, int h, int n0) {

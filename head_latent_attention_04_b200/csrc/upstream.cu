@@ -19,10 +19,13 @@
 //   down-projection [W^DQ | W^DKV] (2112 output features) gives c^Q [N][1536]
 //   and the cache row [c^KV | k_rope] [N][576].  With decode batches the
 //   weight read (30 MB) dominates, so the 112 K-chunks are split over a
-//   cluster of 8 CTAs (17 x 8 = 136 CTAs for one token tile): each CTA
-//   accumulates its K range in TMEM, sends row slices of its partial tile to
-//   the CTA that owns them through distributed shared memory, and each CTA
-//   sums the 8 partials of its 16 rows and writes them.
+//   cluster of 4 CTAs (17 x 4 = 68 CTAs for a token tile of up to 256: one
+//   wave, where clusters of 8 fit only two per GPC and took two or three):
+//   each CTA streams its 28 K-chunks through a ring as deep as shared memory
+//   allows (4 stages at 256 tokens, 11 at 16), accumulates in TMEM, sends row
+//   slices of its partial tile to the CTA that owns them through distributed
+//   shared memory, and each CTA sums the 4 partials of its 32 rows and
+//   writes them.
 #include "mla_internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -244,14 +247,17 @@ q_up_absorb_kernel(const __grid_constant__ CUtensorMap tm_uq, const __grid_const
 }
 
 // ----------------------------------------------------------------- fused qkv_a_proj
-constexpr int kSplit = 8;                    // CTAs of a cluster, one K range each
+constexpr int kSplit = 4;                    // CTAs of a cluster, one K range each
 constexpr int kQkvChunks = kDimE / 64;       // 112
-constexpr int kQkvStages = 4;
+constexpr int kQkvMaxStages = 12;
+constexpr int kQkvRingBudget = 200 * 1024;   // the ring takes as many stages as fit (at most 12)
+constexpr int kQkvT = 256;                   // token tile
+constexpr int kRowsPer = 128 / kSplit;       // 32 output rows reduced and written by each CTA
 
 struct QkvParams {
   __nv_bfloat16* c_q;    // [N][1536]
   __nv_bfloat16* kv_a;   // [N][576]
-  int n_tokens, bn;
+  int n_tokens, bn, stages, region;   // region: bytes of the ring / receive area before the barriers
 };
 
 __global__ void __cluster_dims__(1, 1, kSplit) __launch_bounds__(128, 1)
@@ -259,24 +265,24 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
                   const QkvParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int bn = p.bn;
+  const int bn = p.bn, S = p.stages;
   const int stage = kA + bn * 128;
   uint8_t* ring = smem;                    // later: the partial slices received from the cluster
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kQkvStages * stage);
-  uint64_t* empty = full + kQkvStages;
-  uint64_t* done = empty + kQkvStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.region);
+  uint64_t* empty = full + kQkvMaxStages;
+  uint64_t* done = empty + kQkvMaxStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const int mt = blockIdx.x, n0 = blockIdx.y * bn;
-  const uint32_t cols = bn <= 32 ? 32u : bn <= 64 ? 64u : 128u;
-  constexpr int kPer = kQkvChunks / kSplit;   // 14 K chunks per CTA
+  const uint32_t cols = bn <= 32 ? 32u : bn <= 64 ? 64u : bn <= 128 ? 128u : 256u;
+  constexpr int kPer = kQkvChunks / kSplit;   // 28 K chunks per CTA
   const int kc0 = (int)rank * kPer;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQkvStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -300,8 +306,8 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
 
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < kPer; ++i) {
-      const int s = i % kQkvStages;
-      if (i >= kQkvStages && !mbar_wait(&empty[s], ((i / kQkvStages) - 1) & 1, abort_flag)) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1, abort_flag)) {
         *abort_flag = 1;
         break;
       }
@@ -313,8 +319,8 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = idesc_bf16(128, bn, 0, 0);
     for (int i = 0; i < kPer; ++i) {
-      const int s = i % kQkvStages;
-      if (!mbar_wait(&full[s], (i / kQkvStages) & 1, abort_flag)) {
+      const int s = i % S;
+      if (!mbar_wait(&full[s], (i / S) & 1, abort_flag)) {
         *abort_flag = 1;
         break;
       }
@@ -333,13 +339,11 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
   tc_fence_after();
   cluster_sync();   // every CTA of the cluster is done with its ring before slices land in it
 
-  // ---------------- exchange: row m of the partial tile goes to CTA m / 16, slot `rank`
-  // receive area: [kSplit slots][16 rows][bn] fp32 in the (drained) ring
+  // ---------------- exchange: row m of the partial tile goes to CTA m / 32 (= the warp), slot `rank`
+  // receive area: [kSplit slots][32 rows][bn] fp32 in the (drained) ring
   float* recv = reinterpret_cast<float*>(ring);
   if (ok) {
-    const int m = warp * 32 + lane;
-    const uint32_t owner = (uint32_t)(m >> 4);
-    const uint32_t dst = mapa(smem_u32(recv + ((size_t)rank * 16 + (m & 15)) * bn), owner);
+    const uint32_t dst = mapa(smem_u32(recv + ((size_t)rank * kRowsPer + lane) * bn), (uint32_t)warp);
     for (int c = 0; c < bn; c += 32) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
@@ -355,25 +359,28 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
   tc_fence_before();
   cluster_sync();   // every slice has landed (release / acquire at cluster scope)
   if (ok) {
-    // thread t: token n0 + t, rows 16 rank .. 16 rank + 15 of the tile
-    for (int t = threadIdx.x; t < bn; t += 128) {
+    // thread t: token n0 + t, rows 32 rank .. 32 rank + 31 of the tile, in two halves of 16
+    const int f_base = mt * 128 + kRowsPer * (int)rank;   // first output feature of this slice
+    for (int t = threadIdx.x; t < bn && f_base < kQkvOut; t += 128) {
       const int n = n0 + t;
       if (n >= p.n_tokens) continue;
-      float acc[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll 1
-      for (int s = 0; s < kSplit; ++s)
+      for (int hf = 0; hf < 2; ++hf) {
+        float acc[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] += recv[((size_t)s * 16 + i) * bn + t];
-      const int f0 = mt * 128 + 16 * (int)rank;   // first output feature of this slice
-      if (f0 >= kQkvOut) continue;
-      uint32_t pk[8];
+        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll 1
+        for (int sl = 0; sl < kSplit; ++sl)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(acc[2 * i], acc[2 * i + 1]);
-      __nv_bfloat16* dst = f0 < kQLora ? p.c_q + (size_t)n * kQLora + f0 : p.kv_a + (size_t)n * kKvA + (f0 - kQLora);
-      reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          for (int i = 0; i < 16; ++i) acc[i] += recv[((size_t)sl * kRowsPer + 16 * hf + i) * bn + t];
+        const int f0 = f_base + 16 * hf;
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) pk[i] = pack_bf16(acc[2 * i], acc[2 * i + 1]);
+        __nv_bfloat16* dst = f0 < kQLora ? p.c_q + (size_t)n * kQLora + f0 : p.kv_a + (size_t)n * kKvA + (f0 - kQLora);
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
     }
   }
   tc_fence_before();
@@ -454,8 +461,9 @@ mla_status_t launch_q_up_absorb(const void* c_q, const void* w_uq, const void* w
 }
 
 mla_status_t launch_qkv_a_proj(const void* x, const void* w, void* c_q, void* kv_a, int n_tokens, void* stream) {
-  int tiles = 1;
-  const int bn = tile_tokens(n_tokens, &tiles);
+  const int tiles = (n_tokens + kQkvT - 1) / kQkvT;
+  const int per = (n_tokens + tiles - 1) / tiles;
+  const int bn = ((per + 15) / 16) * 16;    // near-equal token tiles of at most 256, multiples of 16
   CUtensorMap tw, tx;
   {
     const uint64_t dims[2] = {kDimE, kQkvOut};
@@ -471,10 +479,15 @@ mla_status_t launch_qkv_a_proj(const void* x, const void* w, void* c_q, void* kv
     mla_status_t st = encode_tmap_bf16(&tx, x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != MLA_OK) return st;
   }
-  const int ring = kQkvStages * (kA + bn * 128);
-  const int recv = kSplit * 16 * bn * 4;
-  const int smem = 1024 + (ring > recv ? ring : recv) + 256;
-  QkvParams p{static_cast<__nv_bfloat16*>(c_q), static_cast<__nv_bfloat16*>(kv_a), n_tokens, bn};
+  const int stage = kA + bn * 128;
+  int stages = kQkvRingBudget / stage;
+  if (stages > kQkvMaxStages) stages = kQkvMaxStages;
+  if (stages > kQkvChunks / kSplit) stages = kQkvChunks / kSplit;
+  const int ring = stages * stage;
+  const int recv = kSplit * kRowsPer * bn * 4;
+  const int region = ring > recv ? ring : recv;
+  const int smem = 1024 + region + 256;
+  QkvParams p{static_cast<__nv_bfloat16*>(c_q), static_cast<__nv_bfloat16*>(kv_a), n_tokens, bn, stages, region};
   cudaError_t e = upstream_attrs(0, 0);
   if (e == cudaSuccess) {
     e = launch_pdl(qkv_a_proj_kernel, dim3((kQkvOut + 127) / 128, tiles, kSplit), dim3(128), smem, stream, tw, tx, p);

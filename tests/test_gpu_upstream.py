@@ -39,7 +39,7 @@ def test_q_up_absorb_matches_oracle(mla, N, H):
     check_out(q_lat, want)
 
 
-@pytest.mark.parametrize("N", [1, 32, 128, 130, 256])
+@pytest.mark.parametrize("N", [1, 32, 128, 130, 256, 257, 600])
 def test_qkv_a_proj_matches_oracle(mla, N):
     g = torch.Generator().manual_seed(N + 7)
     x = _bf16((N, 7168), 1.0, g)
