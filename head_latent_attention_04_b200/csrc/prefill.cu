@@ -21,12 +21,14 @@
 //   through a three-stage ring (two CTAs per SM); the TMA-store epilogue
 //   writes K or V [T][h][128] bf16.
 // prefill_attn_kernel: one CTA per (128-query tile, head).  Warp 0 stages
-//   the Q tile once and K / k_rope / V tiles of 128 keys through a two-stage
-//   ring; warp 1 issues S = Q K^T (M = 128 queries, N = 128 keys, K = 192:
+//   the Q tile once and K + k_rope and V tiles of 128 keys through two
+//   two-stage rings (a K stage is released by its QK product, a V stage by
+//   its PV product); warp 1 issues S = Q K^T (M = 128 queries, N = 128 keys, K = 192:
 //   8 MMAs on K, 4 on k_rope) into a single S buffer; warp 2 issues
 //   O += P V (M = 128, N = 128, K = 128 keys: 8 MMAs) from two P buffers;
-//   warps 3-6 run the online softmax, one thread per query row (TMEM lane
-//   quarter = warp % 4), with the causal mask on the diagonal tiles and a
+//   warps 3-10 run the online softmax, two threads per query row (TMEM lane
+//   quarter = warp % 4, one 64-key half each, their maxima and sums combined
+//   through shared memory), with the causal mask on the diagonal tiles and a
 //   lazy reference maximum, and write the normalised rows.
 // TMEM (512 columns): S [0,128) fp32, P [128,192) and [192,256) bf16 pairs,
 // O [256,384) fp32.
@@ -163,22 +165,27 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
 }
 
 // ----------------------------------------------------------------- causal attention
-constexpr int kAttThreads = 224;            // 7 warps
-constexpr int kSoftWarp0 = 3;
+constexpr int kAttThreads = 352;            // 11 warps
+constexpr int kSoftWarp0 = 3;               // softmax: warps 3 .. 10, two per TMEM lane quarter
+constexpr int kSoftWarps = 8;
 constexpr int kKStageBytes = 3 * kChunk;    // K (two 64-d chunks) + k_rope (one 64-col chunk)
 constexpr int kVStageBytes = 2 * kChunk;    // V as two 64-v chunks (MN-major B)
 constexpr int kStageBytes = kKStageBytes + kVStageBytes;   // 80 KB
 constexpr int kAttStages = 2;
 constexpr int kOffQ = 0;                                   // Q: q_nope (two chunks) + q_rope (one)
 constexpr int kOffStages = 3 * kChunk;
-constexpr int kOffBar = kOffStages + kAttStages * kStageBytes;
+constexpr int kOffPMax = kOffStages + kAttStages * kStageBytes;   // fp32 [2 tiles][2 halves][128] half-row maxima
+constexpr int kOffLSum = kOffPMax + 4 * kTile * 4;                  // fp32 [2 halves][128] half-row sums
+constexpr int kOffBar = kOffLSum + 2 * kTile * 4;
 constexpr uint32_t kTS = 0, kTP = 128, kTO = 256, kTCols = 512;
 constexpr float kRescale = 8.0f;            // log2 units
 
 struct AttBars {
-  uint64_t q_full, kv_full[kAttStages], kv_empty[kAttStages];
+  uint64_t q_full, k_full[kAttStages], k_empty[kAttStages], v_full[kAttStages], v_empty[kAttStages];
   uint64_t s_full, s_read, p_full[2], o_full[2], o_done;
   uint64_t qk_done, pv_done;
+  uint64_t pmax[2][4];   // the two softmax warps of lane quarter q posted their tile-b half-row maxima
+  uint64_t lsum[4];      // ... and, at the end, their half-row sums
   uint32_t tmem_base;
   int abort;
 };
@@ -219,13 +226,20 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kAttStages; ++s) {
-      mbar_init(&bars->kv_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->k_empty[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->v_empty[s], 1);
     }
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_read, 4);
-    mbar_init(&bars->p_full[0], 4);
-    mbar_init(&bars->p_full[1], 4);
+    mbar_init(&bars->s_read, kSoftWarps);
+    mbar_init(&bars->p_full[0], kSoftWarps);
+    mbar_init(&bars->p_full[1], kSoftWarps);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bars->pmax[0][q], 2);
+      mbar_init(&bars->pmax[1][q], 2);
+      mbar_init(&bars->lsum[q], 2);
+    }
     mbar_init(&bars->o_full[0], 1);
     mbar_init(&bars->o_full[1], 1);
     mbar_init(&bars->o_done, 1);
@@ -252,10 +266,13 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
       tma_load_3d(sQ, &tm_qn, &bars->q_full, 0, h, q0);             // rows past s: zero fill
       tma_load_3d(sQ + kChunk, &tm_qn, &bars->q_full, 64, h, q0);
       tma_load_3d(sQ + 2 * kChunk, &tm_qr, &bars->q_full, 0, h, q0);
-      int j = 0;
-      for (; j < n_tiles; ++j) {
+      // K (with k_rope) and V of a tile are separate rings: a K stage is free
+      // once its QK product completed, a V stage once its PV product did, so
+      // the next K tile loads a whole softmax earlier than a joint stage would.
+      int jk = 0, jv = 0;   // tiles whose K / V loads were issued
+      for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kAttStages;
-        if (j >= kAttStages && !mbar_wait(&bars->kv_empty[s], ((j / kAttStages) - 1) & 1, abort_flag)) {
+        if (j >= kAttStages && !mbar_wait(&bars->k_empty[s], ((j / kAttStages) - 1) & 1, abort_flag)) {
           *abort_flag = 1;
           break;
         }
@@ -266,17 +283,26 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
           blk[q] = (b < 0 || b >= p.num_blocks) ? 0 : b;
         }
         uint8_t* st = sKV + s * kStageBytes;
-        mbar_arrive_expect_tx(&bars->kv_full[s], kStageBytes);
-        tma_load_3d(st, &tm_k, &bars->kv_full[s], 0, h, j * kTile);          // keys past T: zero fill
-        tma_load_3d(st + kChunk, &tm_k, &bars->kv_full[s], 64, h, j * kTile);
-        tma_load_3d(st + 2 * kChunk, &tm_pool, &bars->kv_full[s], 512, 0, blk[0]);   // k_rope, keys 0..63
-        tma_load_3d(st + 2 * kChunk + kChunk / 2, &tm_pool, &bars->kv_full[s], 512, 0, blk[1]);
-        tma_load_3d(st + kKStageBytes, &tm_v, &bars->kv_full[s], 0, h, j * kTile);
-        tma_load_3d(st + kKStageBytes + kChunk, &tm_v, &bars->kv_full[s], 64, h, j * kTile);
+        mbar_arrive_expect_tx(&bars->k_full[s], kKStageBytes);
+        tma_load_3d(st, &tm_k, &bars->k_full[s], 0, h, j * kTile);          // keys past T: zero fill
+        tma_load_3d(st + kChunk, &tm_k, &bars->k_full[s], 64, h, j * kTile);
+        tma_load_3d(st + 2 * kChunk, &tm_pool, &bars->k_full[s], 512, 0, blk[0]);   // k_rope, keys 0..63
+        tma_load_3d(st + 2 * kChunk + kChunk / 2, &tm_pool, &bars->k_full[s], 512, 0, blk[1]);
+        jk = j + 1;
+        if (j >= kAttStages && !mbar_wait(&bars->v_empty[s], ((j / kAttStages) - 1) & 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars->v_full[s], kVStageBytes);
+        tma_load_3d(st + kKStageBytes, &tm_v, &bars->v_full[s], 0, h, j * kTile);
+        tma_load_3d(st + kKStageBytes + kChunk, &tm_v, &bars->v_full[s], 64, h, j * kTile);
+        jv = j + 1;
       }
       // every issued load must land before the CTA exits
-      for (int k = j - 1; k >= 0 && k >= j - kAttStages; --k)
-        mbar_drain(&bars->kv_full[k % kAttStages], (k / kAttStages) & 1);
+      for (int k = jk - 1; k >= 0 && k >= jk - kAttStages; --k)
+        mbar_drain(&bars->k_full[k % kAttStages], (k / kAttStages) & 1);
+      for (int k = jv - 1; k >= 0 && k >= jv - kAttStages; --k)
+        mbar_drain(&bars->v_full[k % kAttStages], (k / kAttStages) & 1);
       mbar_drain(&bars->q_full, 0);
     }
   } else if (warp == 1) {
@@ -287,7 +313,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
       const uint32_t q_addr = smem_u32(sQ);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kAttStages;
-        if (!mbar_wait(&bars->kv_full[s], (j / kAttStages) & 1, abort_flag) ||
+        if (!mbar_wait(&bars->k_full[s], (j / kAttStages) & 1, abort_flag) ||
             (j > 0 && !mbar_wait(&bars->s_read, (j - 1) & 1, abort_flag))) {
           ok = false;
           break;
@@ -300,6 +326,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
           mma_ss(tmem + kTS, sdesc(q_addr + off, 16, 1024, kSwizzle128B), sdesc(k_addr + off, 16, 1024, kSwizzle128B),
                  idesc, t != 0);
         }
+        mma_commit(&bars->k_empty[s]);
         mma_commit(&bars->s_full);
       }
       if (!ok) *abort_flag = 1;
@@ -313,7 +340,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kAttStages;
-        if (!mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag)) {
+        if (!mbar_wait(&bars->v_full[s], (j / kAttStages) & 1, abort_flag) ||
+            !mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -323,7 +351,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
         for (int kk = 0; kk < 8; ++kk)   // 128 keys in steps of 16
           mma_ts(tmem + kTO, tmem + kTP + 64 * (j & 1) + 8 * kk,
                  sdesc(v_addr + kk * 2048, kChunk, 1024, kSwizzle128B), idesc, (j | kk) != 0);
-        mma_commit(&bars->kv_empty[s]);
+        mma_commit(&bars->v_empty[s]);
         mma_commit(&bars->o_full[j & 1]);
       }
       if (ok) mma_commit(&bars->o_done);
@@ -332,34 +360,47 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
       mbar_drain(&bars->pv_done, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax (4 warps, one thread per query)
+    // ------------------------------------------------------------ softmax (8 warps)
+    // Thread = (query row r, key half c): keys [64c, 64c + 64) of each tile and
+    // output columns [64c, 64c + 64).  The two halves of a row combine their
+    // maxima per tile and their sums at the end through shared memory, in the
+    // same order, so both take the same rescaling decisions.
     const int quarter = warp & 3;
+    const int c = (warp - kSoftWarp0) >> 2;
     const int r = quarter * 32 + lane;                 // query row of the tile = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    float* s_pmax = reinterpret_cast<float*>(smem + kOffPMax);
+    float* s_lsum = reinterpret_cast<float*>(smem + kOffLSum);
     const int qpos = pos0 + q0 + r;                    // position of this query (keys <= qpos visible)
     const float sl2 = p.scale_log2;
     float m_ref = -CUDART_INF_F, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
+      const int b = j & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full, j & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      uint32_t v[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + kTS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
+      uint32_t v[64];
+      tmem_ld32(tmem + lane_addr + kTS + 64 * c, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld32(tmem + lane_addr + kTS + 64 * c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_read);
-      // causal mask: key j * 128 + c is visible iff <= qpos (which also excludes keys >= T)
-      const int vis = qpos - j * kTile;                // columns [0, vis] visible
-      float mx = -CUDART_INF_F;
+      // causal mask: key j * 128 + 64c + k is visible iff <= qpos (which also excludes keys >= T)
+      const int vis = qpos - j * kTile - 64 * c;       // columns [0, vis] of this half visible
+      float mloc = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float x = __uint_as_float(v[c]) * sl2;
-        if (c > vis) x = -CUDART_INF_F;
-        v[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+      for (int k = 0; k < 64; ++k) {
+        float x = __uint_as_float(v[k]) * sl2;
+        if (k > vis) x = -CUDART_INF_F;
+        v[k] = __float_as_uint(x);
+        mloc = fmaxf(mloc, x);
       }
+      s_pmax[(b * 2 + c) * kTile + r] = mloc;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->pmax[b][quarter]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->pmax[b][quarter], (j >> 1) & 1, abort_flag))) { ok = false; break; }
+      const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kTile + r]);
       const float m_new = fmaxf(m_ref, mx);
       const bool move = (m_ref == -CUDART_INF_F) ? (m_new != -CUDART_INF_F) : (m_new > m_ref + kRescale);
       float alpha = 1.f;
@@ -368,10 +409,10 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
         m_ref = m_new;
       }
       const float nb = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
-      uint32_t pk[64];
+      uint32_t pk[32];
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
+      for (int k = 0; k < 32; ++k) {
         const float e0 = ex2f(__uint_as_float(v[2 * k]) + nb), e1 = ex2f(__uint_as_float(v[2 * k + 1]) + nb);
         pk[k] = pack_bf16(e0, e1);
         ps[k & 3] += e0 + e1;
@@ -383,7 +424,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
         break;
       }
       if (__any_sync(0xffffffffu, move && j > 0)) {
-        // rescale O: the PV product of tile j - 1 must have landed
+        // rescale this half's O columns: the PV product of tile j - 1 must have landed
         if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag))) {
           ok = false;
           break;
@@ -391,18 +432,17 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
         tc_fence_after();
         const float a = (move && j > 0) ? alpha : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t o[32];
-          tmem_ld32(tmem + lane_addr + kTO + 32 * c, o);
+          tmem_ld32(tmem + lane_addr + kTO + 64 * c + 32 * cc, o);
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
-          tmem_st32(tmem + lane_addr + kTO + 32 * c, o);
+          tmem_st32(tmem + lane_addr + kTO + 64 * c + 32 * cc, o);
         }
         tmem_st_wait();
       }
-      tmem_st32(tmem + lane_addr + kTP + 64 * (j & 1), *reinterpret_cast<uint32_t(*)[32]>(pk));
-      tmem_st32(tmem + lane_addr + kTP + 64 * (j & 1) + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      tmem_st32(tmem + lane_addr + kTP + 64 * (j & 1) + 32 * c, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -410,16 +450,23 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
     }
     if (ok && !__all_sync(0xffffffffu, mbar_wait(&bars->o_done, 0, abort_flag))) ok = false;
     if (ok) {
+      s_lsum[c * kTile + r] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->lsum[quarter]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->lsum[quarter], 0, abort_flag))) ok = false;
+    }
+    if (ok) {
       tc_fence_after();
+      l_run = s_lsum[r] + s_lsum[kTile + r];           // same order in both halves
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const int q = q0 + r;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_addr + kTO + 32 * c, o);
+        tmem_ld32(tmem + lane_addr + kTO + 64 * c + 32 * cc, o);
         tmem_ld_wait();
         if (q < p.s) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)q * p.n_heads + h) * 128 + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)q * p.n_heads + h) * 128 + 64 * c + 32 * cc);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             dst[k] = make_uint4(pack_bf16(__uint_as_float(o[8 * k]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
@@ -428,7 +475,8 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
                                 pack_bf16(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
         }
       }
-      if (q < p.s && p.lse) p.lse[(size_t)q * p.n_heads + h] = l_run > 0.f ? (m_ref + __log2f(l_run)) * 0.6931471805599453f : -CUDART_INF_F;
+      if (c == 0 && q < p.s && p.lse)
+        p.lse[(size_t)q * p.n_heads + h] = l_run > 0.f ? (m_ref + __log2f(l_run)) * 0.6931471805599453f : -CUDART_INF_F;
     } else {
       *abort_flag = 1;
     }

@@ -19,13 +19,14 @@
 //   down-projection [W^DQ | W^DKV] (2112 output features) gives c^Q [N][1536]
 //   and the cache row [c^KV | k_rope] [N][576].  With decode batches the
 //   weight read (30 MB) dominates, so the 112 K-chunks are split over a
-//   cluster of 4 CTAs (17 x 4 = 68 CTAs for a token tile of up to 256: one
-//   wave, where clusters of 8 fit only two per GPC and took two or three):
-//   each CTA streams its 28 K-chunks through a ring as deep as shared memory
-//   allows (4 stages at 256 tokens, 11 at 16), accumulates in TMEM, sends row
-//   slices of its partial tile to the CTA that owns them through distributed
-//   shared memory, and each CTA sums the 4 partials of its 32 rows and
-//   writes them.
+//   cluster of CTAs: 8 when the tokens fit one tile of 128 (17 x 8 = 136
+//   CTAs), else 4 per tile (17 x 4 x tiles).  Each CTA streams its K-chunks
+//   through a ring of at most 104 KB (3 stages at 128 tokens, 5 at 16), so two
+//   CTAs share an SM and the whole grid is resident; it accumulates in TMEM,
+//   sends row slices of its partial tile to the CTA that owns them through
+//   distributed shared memory, and each CTA sums the partials of its 16 or 32
+//   rows and writes them.  (One CTA per SM with clusters of 8 left a second
+//   wave: a GPC holds only two such clusters.)
 #include "mla_internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -247,12 +248,14 @@ q_up_absorb_kernel(const __grid_constant__ CUtensorMap tm_uq, const __grid_const
 }
 
 // ----------------------------------------------------------------- fused qkv_a_proj
-constexpr int kSplit = 4;                    // CTAs of a cluster, one K range each
+// KS CTAs of a cluster, one K range each: 8 for token tiles of up to 128
+// tokens when the batch has one tile (136 CTAs), 4 when it has more (17 x 4 x
+// tiles CTAs).  Either way the ring stays under half of an SM's shared memory,
+// so two CTAs share an SM and every cluster of the grid is resident at once.
 constexpr int kQkvChunks = kDimE / 64;       // 112
-constexpr int kQkvMaxStages = 12;
-constexpr int kQkvRingBudget = 200 * 1024;   // the ring takes as many stages as fit (at most 12)
-constexpr int kQkvT = 256;                   // token tile
-constexpr int kRowsPer = 128 / kSplit;       // 32 output rows reduced and written by each CTA
+constexpr int kQkvMaxStages = 8;
+constexpr int kQkvRingBudget = 104 * 1024;   // the ring takes as many stages as fit
+constexpr int kQkvT = 128;                   // token tile
 
 struct QkvParams {
   __nv_bfloat16* c_q;    // [N][1536]
@@ -260,7 +263,8 @@ struct QkvParams {
   int n_tokens, bn, stages, region;   // region: bytes of the ring / receive area before the barriers
 };
 
-__global__ void __cluster_dims__(1, 1, kSplit) __launch_bounds__(128, 1)
+template <int KS>
+__global__ void __cluster_dims__(1, 1, KS) __launch_bounds__(128, 1)
 qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                   const QkvParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -277,8 +281,9 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t rank = cluster_ctarank();
   const int mt = blockIdx.x, n0 = blockIdx.y * bn;
-  const uint32_t cols = bn <= 32 ? 32u : bn <= 64 ? 64u : bn <= 128 ? 128u : 256u;
-  constexpr int kPer = kQkvChunks / kSplit;   // 28 K chunks per CTA
+  const uint32_t cols = bn <= 32 ? 32u : bn <= 64 ? 64u : 128u;
+  constexpr int kPer = kQkvChunks / KS;       // K chunks per CTA (14 or 28)
+  constexpr int kRowsPer = 128 / KS;          // output rows reduced and written by each CTA
   const int kc0 = (int)rank * kPer;
 
   if (threadIdx.x == 0) {
@@ -339,11 +344,12 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
   tc_fence_after();
   cluster_sync();   // every CTA of the cluster is done with its ring before slices land in it
 
-  // ---------------- exchange: row m of the partial tile goes to CTA m / 32 (= the warp), slot `rank`
-  // receive area: [kSplit slots][32 rows][bn] fp32 in the (drained) ring
+  // ---------------- exchange: row m of the partial tile goes to CTA m / kRowsPer, slot `rank`
+  // receive area: [KS slots][kRowsPer rows][bn] fp32 in the (drained) ring
   float* recv = reinterpret_cast<float*>(ring);
   if (ok) {
-    const uint32_t dst = mapa(smem_u32(recv + ((size_t)rank * kRowsPer + lane) * bn), (uint32_t)warp);
+    const int m = warp * 32 + lane;
+    const uint32_t dst = mapa(smem_u32(recv + ((size_t)rank * kRowsPer + m % kRowsPer) * bn), (uint32_t)(m / kRowsPer));
     for (int c = 0; c < bn; c += 32) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
@@ -359,18 +365,18 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
   tc_fence_before();
   cluster_sync();   // every slice has landed (release / acquire at cluster scope)
   if (ok) {
-    // thread t: token n0 + t, rows 32 rank .. 32 rank + 31 of the tile, in two halves of 16
+    // thread t: token n0 + t, rows kRowsPer rank .. kRowsPer (rank + 1) - 1 of the tile, 16 at a time
     const int f_base = mt * 128 + kRowsPer * (int)rank;   // first output feature of this slice
     for (int t = threadIdx.x; t < bn && f_base < kQkvOut; t += 128) {
       const int n = n0 + t;
       if (n >= p.n_tokens) continue;
 #pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
+      for (int hf = 0; hf < kRowsPer / 16; ++hf) {
         float acc[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] = 0.f;
 #pragma unroll 1
-        for (int sl = 0; sl < kSplit; ++sl)
+        for (int sl = 0; sl < KS; ++sl)
 #pragma unroll
           for (int i = 0; i < 16; ++i) acc[i] += recv[((size_t)sl * kRowsPer + 16 * hf + i) * bn + t];
         const int f0 = f_base + 16 * hf;
@@ -393,8 +399,9 @@ qkv_a_proj_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constan
 cudaError_t upstream_attrs(int smem_q, int smem_qkv) {
   static cudaError_t e = [=] {
     cudaError_t a = cudaFuncSetAttribute(q_up_absorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
-    cudaError_t b = cudaFuncSetAttribute(qkv_a_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
-    return a != cudaSuccess ? a : b;
+    cudaError_t b = cudaFuncSetAttribute(qkv_a_proj_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    cudaError_t c = cudaFuncSetAttribute(qkv_a_proj_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    return a != cudaSuccess ? a : b != cudaSuccess ? b : c;
   }();
   (void)smem_q;
   (void)smem_qkv;
@@ -463,7 +470,8 @@ mla_status_t launch_q_up_absorb(const void* c_q, const void* w_uq, const void* w
 mla_status_t launch_qkv_a_proj(const void* x, const void* w, void* c_q, void* kv_a, int n_tokens, void* stream) {
   const int tiles = (n_tokens + kQkvT - 1) / kQkvT;
   const int per = (n_tokens + tiles - 1) / tiles;
-  const int bn = ((per + 15) / 16) * 16;    // near-equal token tiles of at most 256, multiples of 16
+  const int bn = ((per + 15) / 16) * 16;    // near-equal token tiles of at most 128, multiples of 16
+  const int ks = tiles == 1 ? 8 : 4;
   CUtensorMap tw, tx;
   {
     const uint64_t dims[2] = {kDimE, kQkvOut};
@@ -482,15 +490,16 @@ mla_status_t launch_qkv_a_proj(const void* x, const void* w, void* c_q, void* kv
   const int stage = kA + bn * 128;
   int stages = kQkvRingBudget / stage;
   if (stages > kQkvMaxStages) stages = kQkvMaxStages;
-  if (stages > kQkvChunks / kSplit) stages = kQkvChunks / kSplit;
   const int ring = stages * stage;
-  const int recv = kSplit * kRowsPer * bn * 4;
+  const int recv = 128 * bn * 4;            // KS slots x (128 / KS) rows x bn fp32
   const int region = ring > recv ? ring : recv;
   const int smem = 1024 + region + 256;
   QkvParams p{static_cast<__nv_bfloat16*>(c_q), static_cast<__nv_bfloat16*>(kv_a), n_tokens, bn, stages, region};
   cudaError_t e = upstream_attrs(0, 0);
   if (e == cudaSuccess) {
-    e = launch_pdl(qkv_a_proj_kernel, dim3((kQkvOut + 127) / 128, tiles, kSplit), dim3(128), smem, stream, tw, tx, p);
+    const dim3 grid((kQkvOut + 127) / 128, tiles, ks);
+    e = ks == 8 ? launch_pdl(qkv_a_proj_kernel<8>, grid, dim3(128), smem, stream, tw, tx, p)
+                : launch_pdl(qkv_a_proj_kernel<4>, grid, dim3(128), smem, stream, tw, tx, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "qkv_a_proj launch: %s", cudaGetErrorString(e));
