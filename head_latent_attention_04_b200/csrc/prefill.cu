@@ -21,17 +21,18 @@
 //   through a three-stage ring (two CTAs per SM); the TMA-store epilogue
 //   writes K or V [T][h][128] bf16.
 // prefill_attn_kernel: one CTA per (128-query tile, head).  Warp 0 stages
-//   the Q tile once and K + k_rope and V tiles of 128 keys through two
-//   two-stage rings (a K stage is released by its QK product, a V stage by
-//   its PV product); warp 1 issues S = Q K^T (M = 128 queries, N = 128 keys, K = 192:
-//   8 MMAs on K, 4 on k_rope) into a single S buffer; warp 2 issues
+//   K + k_rope and V tiles of 128 keys through a three-stage and a two-stage
+//   ring (a K stage is released by its QK product, a V stage by its PV
+//   product); the softmax warps put the Q tile into TMEM once; warp 1 issues
+//   S = Q K^T (M = 128 queries, N = 128 keys, K = 192: 8 MMAs on K, 4 on
+//   k_rope, A = Q from TMEM) into a single S buffer; warp 2 issues
 //   O += P V (M = 128, N = 128, K = 128 keys: 8 MMAs) from two P buffers;
 //   warps 3-10 run the online softmax, two threads per query row (TMEM lane
 //   quarter = warp % 4, one 64-key half each, their maxima and sums combined
 //   through shared memory), with the causal mask on the diagonal tiles and a
 //   lazy reference maximum, and write the normalised rows.
 // TMEM (512 columns): S [0,128) fp32, P [128,192) and [192,256) bf16 pairs,
-// O [256,384) fp32.
+// O [256,384) fp32, Q [384,480) bf16 pairs.
 #include "mla_internal.h"
 #include "ptx.cuh"
 #include "tmap.h"
@@ -168,20 +169,19 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
 constexpr int kAttThreads = 352;            // 11 warps
 constexpr int kSoftWarp0 = 3;               // softmax: warps 3 .. 10, two per TMEM lane quarter
 constexpr int kSoftWarps = 8;
-constexpr int kKStageBytes = 3 * kChunk;    // K (two 64-d chunks) + k_rope (one 64-col chunk)
-constexpr int kVStageBytes = 2 * kChunk;    // V as two 64-v chunks (MN-major B)
-constexpr int kStageBytes = kKStageBytes + kVStageBytes;   // 80 KB
-constexpr int kAttStages = 2;
-constexpr int kOffQ = 0;                                   // Q: q_nope (two chunks) + q_rope (one)
-constexpr int kOffStages = 3 * kChunk;
-constexpr int kOffPMax = kOffStages + kAttStages * kStageBytes;   // fp32 [2 tiles][2 halves][128] half-row maxima
+constexpr int kKStageBytes = 3 * kChunk;    // K (two 64-d chunks) + k_rope (one 64-col chunk), 48 KB
+constexpr int kVStageBytes = 2 * kChunk;    // V as two 64-v chunks (MN-major B), 32 KB
+constexpr int kKStages = 3, kVStages = 2;
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKStages * kKStageBytes;
+constexpr int kOffPMax = kOffV + kVStages * kVStageBytes;          // fp32 [2 tiles][2 halves][128] half-row maxima
 constexpr int kOffLSum = kOffPMax + 4 * kTile * 4;                  // fp32 [2 halves][128] half-row sums
 constexpr int kOffBar = kOffLSum + 2 * kTile * 4;
-constexpr uint32_t kTS = 0, kTP = 128, kTO = 256, kTCols = 512;
+constexpr uint32_t kTS = 0, kTP = 128, kTO = 256, kTQ = 384, kTCols = 512;   // Q: 96 columns of bf16 pairs
 constexpr float kRescale = 8.0f;            // log2 units
 
 struct AttBars {
-  uint64_t q_full, k_full[kAttStages], k_empty[kAttStages], v_full[kAttStages], v_empty[kAttStages];
+  uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t s_full, s_read, p_full[2], o_full[2], o_done;
   uint64_t qk_done, pv_done;
   uint64_t pmax[2][4];   // the two softmax warps of lane quarter q posted their tile-b half-row maxima
@@ -192,6 +192,8 @@ struct AttBars {
 constexpr int kAttSmem = kOffBar + (int)sizeof(AttBars) + 1024;
 
 struct AttParams {
+  const __nv_bfloat16* q_nope;   // [s][H][128]
+  const __nv_bfloat16* q_rope;   // [s][H][64]
   const int32_t* block_row;
   __nv_bfloat16* out;      // [s][H][128]
   float* lse;              // [s][H] or null
@@ -206,13 +208,12 @@ __device__ __forceinline__ float ex2f(float x) {
 }
 
 __global__ void __launch_bounds__(kAttThreads, 1)
-prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qr,
-                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_pool, const AttParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + kOffQ;
-  uint8_t* sKV = smem + kOffStages;
+  uint8_t* sK = smem + kOffK;
+  uint8_t* sV = smem + kOffV;
   AttBars* bars = reinterpret_cast<AttBars*>(smem + kOffBar);
   int* abort_flag = &bars->abort;
 
@@ -224,10 +225,12 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
   const int n_tiles = (pos0 + last_q) / kTile + 1;        // key tiles up to the causal limit
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < kAttStages; ++s) {
+    mbar_init(&bars->q_full, kSoftWarps);   // Q rows stored into TMEM by the softmax warps
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -262,17 +265,13 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bars->q_full, 3 * kChunk);
-      tma_load_3d(sQ, &tm_qn, &bars->q_full, 0, h, q0);             // rows past s: zero fill
-      tma_load_3d(sQ + kChunk, &tm_qn, &bars->q_full, 64, h, q0);
-      tma_load_3d(sQ + 2 * kChunk, &tm_qr, &bars->q_full, 0, h, q0);
       // K (with k_rope) and V of a tile are separate rings: a K stage is free
       // once its QK product completed, a V stage once its PV product did, so
       // the next K tile loads a whole softmax earlier than a joint stage would.
       int jk = 0, jv = 0;   // tiles whose K / V loads were issued
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kAttStages;
-        if (j >= kAttStages && !mbar_wait(&bars->k_empty[s], ((j / kAttStages) - 1) & 1, abort_flag)) {
+        const int s = j % kKStages, sv = j % kVStages;
+        if (j >= kKStages && !mbar_wait(&bars->k_empty[s], ((j / kKStages) - 1) & 1, abort_flag)) {
           *abort_flag = 1;
           break;
         }
@@ -282,49 +281,47 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
           const int b = pg < p.n_pages ? p.block_row[pg] : 0;
           blk[q] = (b < 0 || b >= p.num_blocks) ? 0 : b;
         }
-        uint8_t* st = sKV + s * kStageBytes;
+        uint8_t* st = sK + s * kKStageBytes;
         mbar_arrive_expect_tx(&bars->k_full[s], kKStageBytes);
         tma_load_3d(st, &tm_k, &bars->k_full[s], 0, h, j * kTile);          // keys past T: zero fill
         tma_load_3d(st + kChunk, &tm_k, &bars->k_full[s], 64, h, j * kTile);
         tma_load_3d(st + 2 * kChunk, &tm_pool, &bars->k_full[s], 512, 0, blk[0]);   // k_rope, keys 0..63
         tma_load_3d(st + 2 * kChunk + kChunk / 2, &tm_pool, &bars->k_full[s], 512, 0, blk[1]);
         jk = j + 1;
-        if (j >= kAttStages && !mbar_wait(&bars->v_empty[s], ((j / kAttStages) - 1) & 1, abort_flag)) {
+        if (j >= kVStages && !mbar_wait(&bars->v_empty[sv], ((j / kVStages) - 1) & 1, abort_flag)) {
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(&bars->v_full[s], kVStageBytes);
-        tma_load_3d(st + kKStageBytes, &tm_v, &bars->v_full[s], 0, h, j * kTile);
-        tma_load_3d(st + kKStageBytes + kChunk, &tm_v, &bars->v_full[s], 64, h, j * kTile);
+        uint8_t* sv_st = sV + sv * kVStageBytes;
+        mbar_arrive_expect_tx(&bars->v_full[sv], kVStageBytes);
+        tma_load_3d(sv_st, &tm_v, &bars->v_full[sv], 0, h, j * kTile);
+        tma_load_3d(sv_st + kChunk, &tm_v, &bars->v_full[sv], 64, h, j * kTile);
         jv = j + 1;
       }
       // every issued load must land before the CTA exits
-      for (int k = jk - 1; k >= 0 && k >= jk - kAttStages; --k)
-        mbar_drain(&bars->k_full[k % kAttStages], (k / kAttStages) & 1);
-      for (int k = jv - 1; k >= 0 && k >= jv - kAttStages; --k)
-        mbar_drain(&bars->v_full[k % kAttStages], (k / kAttStages) & 1);
-      mbar_drain(&bars->q_full, 0);
+      for (int k = jk - 1; k >= 0 && k >= jk - kKStages; --k)
+        mbar_drain(&bars->k_full[k % kKStages], (k / kKStages) & 1);
+      for (int k = jv - 1; k >= 0 && k >= jv - kVStages; --k)
+        mbar_drain(&bars->v_full[k % kVStages], (k / kVStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ QK issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, kTile, 0, 0);
       bool ok = mbar_wait(&bars->q_full, 0, abort_flag);
-      const uint32_t q_addr = smem_u32(sQ);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kAttStages;
-        if (!mbar_wait(&bars->k_full[s], (j / kAttStages) & 1, abort_flag) ||
+        const int s = j % kKStages;
+        if (!mbar_wait(&bars->k_full[s], (j / kKStages) & 1, abort_flag) ||
             (j > 0 && !mbar_wait(&bars->s_read, (j - 1) & 1, abort_flag))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sKV + s * kStageBytes);
+        const uint32_t k_addr = smem_u32(sK + s * kKStageBytes);
 #pragma unroll
-        for (int t = 0; t < 12; ++t) {   // K = 192 in steps of 16: chunk t / 4 (nope, nope, rope)
+        for (int t = 0; t < 12; ++t) {   // K = 192 in steps of 16: chunk t / 4 (nope, nope, rope); A = Q from TMEM
           const uint32_t off = (t >> 2) * kChunk + (t & 3) * 32;
-          mma_ss(tmem + kTS, sdesc(q_addr + off, 16, 1024, kSwizzle128B), sdesc(k_addr + off, 16, 1024, kSwizzle128B),
-                 idesc, t != 0);
+          mma_ts(tmem + kTS, tmem + kTQ + 8 * t, sdesc(k_addr + off, 16, 1024, kSwizzle128B), idesc, t != 0);
         }
         mma_commit(&bars->k_empty[s]);
         mma_commit(&bars->s_full);
@@ -339,14 +336,14 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
       const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kAttStages;
-        if (!mbar_wait(&bars->v_full[s], (j / kAttStages) & 1, abort_flag) ||
+        const int s = j % kVStages;
+        if (!mbar_wait(&bars->v_full[s], (j / kVStages) & 1, abort_flag) ||
             !mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sKV + s * kStageBytes + kKStageBytes);
+        const uint32_t v_addr = smem_u32(sV + s * kVStageBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // 128 keys in steps of 16
           mma_ts(tmem + kTO, tmem + kTP + 64 * (j & 1) + 8 * kk,
@@ -373,6 +370,38 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_qn, const __grid_cons
     float* s_lsum = reinterpret_cast<float*>(smem + kOffLSum);
     const int qpos = pos0 + q0 + r;                    // position of this query (keys <= qpos visible)
     const float sl2 = p.scale_log2;
+    {
+      // the tile's query rows into TMEM (A operand of QK): half 0 the q_nope row
+      // (64 columns of bf16 pairs), half 1 the q_rope row (32 columns)
+      const int q = q0 + r;
+      const uint4 zero = make_uint4(0, 0, 0, 0);
+      if (c == 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + ((size_t)q * p.n_heads + h) * 128);
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t v[32];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint4 x = q < p.s ? __ldg(src + 8 * hh + k) : zero;
+            v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+          }
+          tmem_st32(tmem + lane_addr + kTQ + 32 * hh, v);
+        }
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + ((size_t)q * p.n_heads + h) * 64);
+        uint32_t v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint4 x = q < p.s ? __ldg(src + k) : zero;
+          v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+        }
+        tmem_st32(tmem + lane_addr + kTQ + 64, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->q_full);
+    }
     float m_ref = -CUDART_INF_F, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -544,19 +573,18 @@ mla_status_t launch_prefill_up_proj(const void* kv_pool, const int32_t* block_ro
 mla_status_t launch_prefill_attn(const void* q_nope, const void* q_rope, const void* k, const void* v,
                                  const void* kv_pool, const int32_t* block_row, int T, int s, int n_heads,
                                  int num_blocks, float scale, void* out, float* lse, void* stream) {
-  CUtensorMap tqn, tqr, tk, tv, tpool;
-  mla_status_t st = rows_map(&tqn, q_nope, 128, n_heads, s, false);
-  if (st == MLA_OK) st = rows_map(&tqr, q_rope, 64, n_heads, s, false);
-  if (st == MLA_OK) st = rows_map(&tk, k, 128, n_heads, T, false);
+  CUtensorMap tk, tv, tpool;
+  mla_status_t st = rows_map(&tk, k, 128, n_heads, T, false);
   if (st == MLA_OK) st = rows_map(&tv, v, 128, n_heads, T, false);
   if (st == MLA_OK) st = pool_map(&tpool, kv_pool, num_blocks);
   if (st != MLA_OK) return st;
-  AttParams p{block_row, static_cast<__nv_bfloat16*>(out), lse, T, s, n_heads, (T + 63) / 64, num_blocks,
+  AttParams p{static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_rope), block_row,
+              static_cast<__nv_bfloat16*>(out), lse, T, s, n_heads, (T + 63) / 64, num_blocks,
               scale * 1.4426950408889634f};
   cudaError_t e = prefill_attrs();
   if (e == cudaSuccess) {
     e = launch_pdl(prefill_attn_kernel, dim3((s + kTile - 1) / kTile, n_heads), dim3(kAttThreads), kAttSmem, stream,
-                   tqn, tqr, tk, tv, tpool, p);
+                   tk, tv, tpool, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "prefill attention launch: %s", cudaGetErrorString(e));
