@@ -35,3 +35,23 @@ def test_algorithmic_accounting_fp8_weights():
     f8 = bench.algorithmic([4096] * 32, 1, 128, weight_bytes=1)
     assert bf["step_bytes"] - f8["step_bytes"] == 2 * 512 * 128 * 128 - 2 * 4 * 128 * 4
     assert f8["attn_bytes"] == bf["attn_bytes"] and f8["step_flops"] == bf["step_flops"]
+
+
+def test_algorithmic_accounting_fp8_cache():
+    """FP8 latent cache: 656 bytes per cached token (512 codes, 4 fp32 scales,
+    64 bf16 k_rope) instead of 1152; the products are unchanged."""
+    bf = bench.algorithmic([4096] * 32, 1, 128)
+    f8 = bench.algorithmic([4096] * 32, 1, 128, cache_row_bytes=656)
+    assert 656 == 512 + 4 * 4 + 64 * 2
+    assert f8["cache_bytes"] == 32 * 4096 * 656
+    assert bf["attn_bytes"] - f8["attn_bytes"] == 32 * 4096 * (1152 - 656)
+    assert f8["attn_flops"] == bf["attn_flops"]
+
+
+def test_next_path_roofline_picks_the_binding_unit():
+    peaks = {"hbm_gbs": 6545.0, "bf16_tflops": 1630.1, "bf16_tflops_sustained": 1374.1}
+    # 30.3 MB and 7.75 GFLOP: 4.6 us of HBM against 4.8 us of tensor time -> tensor
+    r = bench._roof(7.75e9, 30.3e6, 0.010, peaks, "measured")
+    assert r["bound"] == "tensor" and abs(r["achieved"] - 775.0) < 1e-6 and abs(r["frac"] - 775.0 / 1630.1) < 1e-9
+    r = bench._roof(1e6, 30.3e6, 0.010, peaks, "measured")
+    assert r["bound"] == "hbm" and abs(r["achieved"] - 3030.0) < 1e-6
