@@ -254,3 +254,47 @@ def test_fp8cache_full_size(mla, name, heads):
     check_out(got, ref["out"])
     got_ol = res.o_lat[rows] if heads is None else res.o_lat[rows][:, heads]
     check_out(got_ol, ref["o_lat"])
+
+
+@pytest.mark.parametrize("s_q,H,lens,clusters", [(8, 128, [8, 9, 70, 640], 74), (3, 33, [3, 64, 200, 1000], 6)])
+def test_fp8cache_long_speculation_and_odd_heads(mla, s_q, H, lens, clusters):
+    """s_q up to 8 causal drafts, and a head count that ends inside a TMEM lane quarter."""
+    w = W.make_workload(len(lens), s_q, H, lens, seed=101 + s_q + H, pool="scattered:2")
+    full_check8(mla, w, num_clusters=clusters)
+
+
+def test_fp8cache_stale_lengths_are_rejected(mla):
+    """The FP8 instance checks the device seq_lens against the plan like the bf16 one."""
+    w = W.make_workload(3, 1, 128, [300, 1000, 77], seed=57, pool="scattered:2")
+    pool8 = oracle_pool(w)
+    dev = torch.device("cuda")
+    dec, res = run_fp8(mla, w, pool8, num_clusters=4)
+    assert res.status.item() == 0
+    dec.seq_lens_dev[1] += 1
+    dec.status.zero_()
+    wd = w.to(dev)
+    r = dec.run(wd.q_nope, wd.q_rope, pool8.to(dev), torch.as_tensor(w.block_table, device=dev), wd.w_uk, wd.w_uv)
+    torch.cuda.synchronize()
+    assert r.status.item() == mla.STATUS_BAD_SEQLEN
+    assert torch.all(r.out[1] == 0) and torch.all(torch.isneginf(r.lse[1]))
+    for b in (0, 2):
+        check_out(r.out[b:b + 1], oracle_rows8(w, pool8, b)["out"])
+
+
+def test_fp8cache_wait_time_out_returns_and_recovers(mla):
+    """Bounded waits in the FP8 instance (the widening waits included): with a
+    1 ns bound the kernel gives up with MLA_STATUS_TIMEOUT and returns, and the
+    next call with the default bound matches the oracle."""
+    w = W.make_workload(3, 2, 128, [2000, 70, 600], seed=68, pool="permuted")
+    pool8 = oracle_pool(w)
+    try:
+        mla.set_wait_limit_ns(1)
+        for _ in range(2):
+            _, res = run_fp8(mla, w, pool8, num_clusters=6)
+            assert res.status.item() & mla.STATUS_TIMEOUT
+    finally:
+        mla.set_wait_limit_ns(0)
+    _, res = run_fp8(mla, w, pool8, num_clusters=6)
+    assert res.status.item() == 0
+    for b in range(w.B):
+        check_out(res.out[b * 2:(b + 1) * 2], oracle_rows8(w, pool8, b)["out"])
