@@ -304,7 +304,8 @@ mla_status_t mla_kv_quantize_fp8(const void* kv, const int32_t* slots, int64_t n
   if (n < 0 || num_blocks < 1) return set_error(MLA_ERR_INVALID_ARG, "n must be >= 0 and num_blocks >= 1");
   if (n == 0) return MLA_OK;
   MLA_TRY(check_ptr(kv, "kv"));
-  MLA_TRY(check_ptr(slots, "slots"));
+  if (!slots || (reinterpret_cast<uintptr_t>(slots) & 3u))
+    return set_error(MLA_ERR_INVALID_ARG, "slots is NULL or not 4-byte aligned");
   MLA_TRY(check_ptr(pool_fp8, "pool_fp8"));
   return launch_kv_quantize_fp8(kv, slots, n, pool_fp8, (long long)num_blocks * 64, status, stream);
 }

@@ -268,7 +268,7 @@ mla_status_t mla_decode_attn_fp8cache(const mla_dims_t* dims, const void* q_lat,
  * s = amax / 448, code = E4M3(x * (448 / amax)) rounded to nearest even and
  * saturated (an all-zero block takes s = 1); k_rope is copied.
  *   kv        bf16 [n][576]  rows c_KV (512) | k_rope (64), 16-byte aligned
- *   slots     int32 [n]      destination of row i: block * 64 + row in the block
+ *   slots     int32 [n]      destination of row i: block * 64 + row in the block (4-byte aligned)
  *   pool_fp8  uint8 [num_blocks][64][656]
  *   status    int32 [1] or NULL: MLA_STATUS_BAD_BLOCK when a slot lies outside
  *             the pool (that row is not written); MLA_STATUS_CACHE_RANGE when a
