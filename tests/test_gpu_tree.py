@@ -82,3 +82,19 @@ def test_tree_full_size_mtp_shape():
             continue
         ref = oracle_rows(w, b, draft_masks=masks[b])
         check_out(out[b * 4:(b + 1) * 4], ref["out"])
+
+
+@pytest.mark.parametrize("s_q,lens,clusters", [(2, [2, 65, 300], 4), (4, [4, 200, 4100], 74)])
+def test_non_causal_plan_without_masks(s_q, lens, clusters):
+    """dims->causal = 0 on the plain entry point: every query attends all T_b
+    keys, the drafts included -- the oracle with every draft visible to every
+    query (all mask bits set)."""
+    w = W.make_workload(len(lens), s_q, 128, lens, seed=s_q + 90, pool="scattered:1.5")
+    dec, res = run_gpu(w, num_clusters=clusters, causal=False)
+    assert res.status.item() == 0
+    full = [(1 << s_q) - 1] * s_q
+    for b in range(w.B):
+        ref = oracle_rows(w, b, draft_masks=full)
+        rows = slice(b * s_q, (b + 1) * s_q)
+        check_out(res.out[rows], ref["out"])
+        np.testing.assert_allclose(res.lse[rows].cpu().numpy(), ref["lse"], rtol=0, atol=2e-2)
