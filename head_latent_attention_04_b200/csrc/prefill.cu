@@ -207,6 +207,12 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
 __global__ void __launch_bounds__(kAttThreads, 1)
 prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_pool, const AttParams p) {
@@ -415,21 +421,29 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->s_read);
-      // causal mask: key j * 128 + 64c + k is visible iff <= qpos (which also excludes keys >= T)
+      // causal mask: key j * 128 + 64c + k is visible iff <= qpos (which also
+      // excludes keys >= T); only the tiles that reach past some row's last
+      // visible key take it.  Maxima are taken on the raw scores (the scale is
+      // positive, so the scaled maximum is the same rounded value).
       const int vis = qpos - j * kTile - 64 * c;       // columns [0, vis] of this half visible
-      float mloc = -CUDART_INF_F;
+      const bool full = __all_sync(0xffffffffu, vis >= 63);
+      if (!full) {
 #pragma unroll
-      for (int k = 0; k < 64; ++k) {
-        float x = __uint_as_float(v[k]) * sl2;
-        if (k > vis) x = -CUDART_INF_F;
-        v[k] = __float_as_uint(x);
-        mloc = fmaxf(mloc, x);
+        for (int k = 0; k < 64; ++k)
+          if (k > vis) v[k] = __float_as_uint(-CUDART_INF_F);
       }
+      float mq[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+      for (int k = 0; k < 64; k += 8)
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          mq[a] = max3f(mq[a], __uint_as_float(v[k + 2 * a]), __uint_as_float(v[k + 2 * a + 1]));
+      const float mloc = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       s_pmax[(b * 2 + c) * kTile + r] = mloc;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->pmax[b][quarter]);
       if (!__all_sync(0xffffffffu, mbar_wait(&bars->pmax[b][quarter], (j >> 1) & 1, abort_flag))) { ok = false; break; }
-      const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kTile + r]);
+      const float mx = fmaxf(mloc, s_pmax[(b * 2 + (c ^ 1)) * kTile + r]) * sl2;
       const float m_new = fmaxf(m_ref, mx);
       const bool move = (m_ref == -CUDART_INF_F) ? (m_new != -CUDART_INF_F) : (m_new > m_ref + kRescale);
       float alpha = 1.f;
@@ -438,15 +452,17 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         m_ref = m_new;
       }
       const float nb = (m_ref == -CUDART_INF_F) ? 0.f : -m_ref;
+      const float2 sl2x2 = make_float2(sl2, sl2), nbx2 = make_float2(nb, nb);
       uint32_t pk[32];
-      float ps[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 ps[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
-        const float e0 = ex2f(__uint_as_float(v[2 * k]) + nb), e1 = ex2f(__uint_as_float(v[2 * k + 1]) + nb);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), sl2x2, nbx2);
+        const float e0 = ex2f(x.x), e1 = ex2f(x.y);
         pk[k] = pack_bf16(e0, e1);
-        ps[k & 3] += e0 + e1;
+        ps[k & 1] = __fadd2_rn(ps[k & 1], make_float2(e0, e1));
       }
-      l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      l_run = l_run * alpha + ((ps[0].x + ps[1].x) + (ps[0].y + ps[1].y));
       // P buffer j & 1 is free once the PV product of tile j - 2 completed
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bars->o_full[j & 1], ((j >> 1) - 1) & 1, abort_flag))) {
         ok = false;
