@@ -14,12 +14,13 @@
 // (the s new tokens of a chunk are already in the cache and sit at positions
 // T - s .. T - 1, so a chunk of s < T tokens is chunked prefill).
 //
-// up_proj_kernel: one CTA per (K or V, head, 128-token tile): a swap-AB
-//   tcgen05 GEMM, M = 128 features of the head's W_UK / W_UV slice, N = 128
-//   tokens (two cache pages, read through the block table by TMA from the
-//   (column, row, block) view of the pool), K = 512 latent columns streamed
-//   through a three-stage ring (two CTAs per SM); the TMA-store epilogue
-//   writes K or V [T][h][128] bf16.
+// up_proj_kernel: one CTA per (128-token tile, head) makes both K and V from one
+//   staged c_KV tile: a tcgen05 GEMM with M = 128 tokens (two cache pages, read
+//   through the block table by TMA from the (column, row, block) view of the
+//   pool), N = 256 (the head's 128 W_UK and 128 W_UV features), K = 512 latent
+//   columns streamed through a two-stage ring (two CTAs per SM); tokens on
+//   TMEM lanes, so each thread packs its token's rows in the SW128 layout of
+//   the output boxes and four TMA stores write K and V [T][h][128] bf16.
 // prefill_attn_kernel: one CTA per (128-query tile, head).  Warp 0 stages
 //   K + k_rope and V tiles of 128 keys through a three-stage and a two-stage
 //   ring (a K stage is released by its QK product, a V stage by its PV
@@ -47,29 +48,11 @@ using namespace ptx;
 
 constexpr int kTile = 128;                 // tokens per tile (queries, keys, up-projection)
 constexpr int kChunk = kTile * 128;        // 16 KB: 128 rows x 64 bf16 (SW128)
-constexpr int kUpStages = 3;            // 97 KB: two CTAs per SM, so one's epilogue overlaps the other's loads
-constexpr int kUpStageBytes = 2 * kChunk;  // W chunk (two 64-feature halves) + c_KV chunk
-
-__device__ __forceinline__ void store_rows(uint32_t tmem, uint8_t* s_out, const CUtensorMap* tm_out, int h, int n0) {
-  // TMEM [128 lanes = features][128 columns = tokens] fp32 -> bf16 [token][128] -> one TMA store
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(s_out);
-  const int m = warp * 32 + lane;
-  for (int c = 0; c < kTile; c += 32) {
-    uint32_t r[32];
-    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < 32; ++j) o[(c + j) * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    tma_store_3d(tm_out, s_out, 0, h, n0);
-    bulk_commit();
-    bulk_wait_all<0>();
-  }
-}
+constexpr int kUpStages = 2;            // 97 KB: two CTAs per SM, so one's epilogue overlaps the other's loads
+constexpr int kUpABytes = kChunk;          // c_KV chunk: 128 tokens x 64 latent columns (two pages, SW128)
+constexpr int kUpBBytes = 4 * kChunk / 2;  // W_UK | W_UV chunk: 64 latent rows x 256 features (four SW128 blocks)
+constexpr int kUpStageBytes = kUpABytes + kUpBBytes;
+constexpr int kUpSmem = 1024 + kUpStages * kUpStageBytes + 256;
 
 struct UpParams {
   const int32_t* block_row;   // the sequence's block-table row
@@ -89,9 +72,7 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const bool is_v = blockIdx.x == 1;
-  const int h = blockIdx.y, t0 = blockIdx.z * kTile;
-  const CUtensorMap* tm_w = is_v ? &tm_wv : &tm_wk;
+  const int t0 = blockIdx.x * kTile, h = blockIdx.y;
   constexpr int kChunks = 512 / 64;
 
   if (threadIdx.x == 0) {
@@ -102,11 +83,12 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(tm_w);
+    prefetch_tmap(&tm_wk);
+    prefetch_tmap(&tm_wv);
     prefetch_tmap(&tm_pool);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTile);
+    tmem_alloc(tmem_slot, 2 * kTile);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -131,14 +113,19 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
         break;
       }
       uint8_t* st = smem + s * kUpStageBytes;
+      uint8_t* sb = st + kUpABytes;
       mbar_arrive_expect_tx(&full[s], kUpStageBytes);
-      tma_load_3d(st, tm_w, &full[s], 0, h, kc * 64);                  // features 0..63 (MN-major)
-      tma_load_3d(st + kChunk / 2, tm_w, &full[s], 64, h, kc * 64);    // features 64..127
-      tma_load_3d(st + kChunk, &tm_pool, &full[s], kc * 64, 0, blk[0]);               // tokens 0..63
-      tma_load_3d(st + kChunk + kChunk / 2, &tm_pool, &full[s], kc * 64, 0, blk[1]);  // tokens 64..127
+      tma_load_3d(st, &tm_pool, &full[s], kc * 64, 0, blk[0]);                   // tokens 0..63
+      tma_load_3d(st + kChunk / 2, &tm_pool, &full[s], kc * 64, 0, blk[1]);      // tokens 64..127
+      tma_load_3d(sb, &tm_wk, &full[s], 0, h, kc * 64);                          // K features 0..63
+      tma_load_3d(sb + kChunk / 2, &tm_wk, &full[s], 64, h, kc * 64);            // K features 64..127
+      tma_load_3d(sb + kChunk, &tm_wv, &full[s], 0, h, kc * 64);                 // V features 0..63
+      tma_load_3d(sb + 3 * kChunk / 2, &tm_wv, &full[s], 64, h, kc * 64);        // V features 64..127
     }
   } else if (warp == 1 && lane == 0) {
-    const uint32_t idesc = idesc_bf16(128, kTile, 1, 0);
+    // D[token][K features | V features] += c_KV[token][k] W[k][feature]: M = 128 tokens
+    // (A K-major), N = 256 (B MN-major, four 64-feature blocks 8 KB apart)
+    const uint32_t idesc = idesc_bf16(128, 2 * kTile, 0, 1);
     for (int kc = 0; kc < kChunks; ++kc) {
       const int s = kc % kUpStages;
       if (!mbar_wait(&full[s], (kc / kUpStages) & 1, abort_flag)) {
@@ -146,11 +133,11 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
         break;
       }
       tc_fence_after();
-      const uint32_t a0 = smem_u32(smem + s * kUpStageBytes), b0 = a0 + kChunk;
+      const uint32_t a0 = smem_u32(smem + s * kUpStageBytes), b0 = a0 + kUpABytes;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ss(tmem, sdesc(a0 + kk * 2048, kChunk / 2, 1024, kSwizzle128B),
-               sdesc(b0 + kk * 32, 16, 1024, kSwizzle128B), idesc, (kc | kk) != 0);
+        mma_ss(tmem, sdesc(a0 + kk * 32, 16, 1024, kSwizzle128B),
+               sdesc(b0 + kk * 2048, kChunk / 2, 1024, kSwizzle128B), idesc, (kc | kk) != 0);
       mma_commit(&empty[s]);
     }
     mma_commit(done);
@@ -158,11 +145,45 @@ up_proj_kernel(const __grid_constant__ CUtensorMap tm_wk, const __grid_constant_
   __syncwarp();
   const bool ok = __syncthreads_and(mbar_wait(done, 0, abort_flag) && !*abort_flag);
   tc_fence_after();
-  if (ok) store_rows(tmem, smem, is_v ? &tm_v : &tm_k, h, t0);
+  if (ok) {
+    // TMEM lane = token, column = feature: each thread packs its token's 64-feature
+    // blocks to bf16 in the SW128 layout of the output boxes (the stage memory is
+    // free: every load landed and every product that read it completed)
+    const int r = warp * 32 + lane;
+#pragma unroll 1
+    for (int blkf = 0; blkf < 4; ++blkf) {
+      uint8_t* dst = smem + blkf * kChunk + r * 128;
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + blkf * 64 + hh * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = hh * 4 + c;   // 16-byte chunk of the 128-byte row
+          st_shared_v4(smem_u32(dst + ((chunk ^ (r & 7)) << 4)),
+                       make_uint4(pack_bf16(__uint_as_float(v[8 * c]), __uint_as_float(v[8 * c + 1])),
+                                  pack_bf16(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3])),
+                                  pack_bf16(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5])),
+                                  pack_bf16(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]))));
+        }
+      }
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
+  if (ok && threadIdx.x == 0) {
+    // rows past T are clipped by the stores
+    tma_store_3d(&tm_k, smem, 0, h, t0);
+    tma_store_3d(&tm_k, smem + kChunk, 64, h, t0);
+    tma_store_3d(&tm_v, smem + 2 * kChunk, 0, h, t0);
+    tma_store_3d(&tm_v, smem + 3 * kChunk, 64, h, t0);
+    bulk_commit();
+    bulk_wait_all<0>();
+  }
   __syncwarp();
-  if (warp == 1) tmem_dealloc(tmem, kTile);
+  if (warp == 1) tmem_dealloc(tmem, 2 * kTile);
 }
 
 // ----------------------------------------------------------------- causal attention
@@ -535,8 +556,7 @@ prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
 cudaError_t prefill_attrs() {
   static cudaError_t e = [] {
-    cudaError_t a = cudaFuncSetAttribute(up_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         1024 + kUpStages * kUpStageBytes + 256);
+    cudaError_t a = cudaFuncSetAttribute(up_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUpSmem);
     cudaError_t b = cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem);
     return a != cudaSuccess ? a : b;
   }();
@@ -545,11 +565,11 @@ cudaError_t prefill_attrs() {
 
 // [N][H][F] bf16 viewed as (F, H, N): boxes of 64 features x 128 rows (SW128), or a
 // store box of 128 features x 128 rows (no swizzle).
-mla_status_t rows_map(CUtensorMap* m, const void* base, int F, int H, int N, bool store) {
+mla_status_t rows_map(CUtensorMap* m, const void* base, int F, int H, int N) {
   const uint64_t dims[3] = {(uint64_t)F, (uint64_t)H, (uint64_t)N};
   const uint64_t str[2] = {(uint64_t)F * 2, (uint64_t)H * F * 2};
-  const uint32_t box[3] = {store ? 128u : 64u, 1, (uint32_t)kTile};
-  return encode_tmap_bf16(m, base, 3, dims, str, box, store ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B);
+  const uint32_t box[3] = {64, 1, (uint32_t)kTile};
+  return encode_tmap_bf16(m, base, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // The cache pool as (column, row within the block, block), boxes of 64 columns x 64 rows.
@@ -572,14 +592,14 @@ mla_status_t launch_prefill_up_proj(const void* kv_pool, const int32_t* block_ro
   mla_status_t st = encode_tmap_bf16(&twk, w_uk, 3, wdims, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st == MLA_OK) st = encode_tmap_bf16(&twv, w_uv, 3, wdims, wstr, wbox, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st == MLA_OK) st = pool_map(&tpool, kv_pool, num_blocks);
-  if (st == MLA_OK) st = rows_map(&tk, k_out, 128, n_heads, T, true);
-  if (st == MLA_OK) st = rows_map(&tv, v_out, 128, n_heads, T, true);
+  if (st == MLA_OK) st = rows_map(&tk, k_out, 128, n_heads, T);
+  if (st == MLA_OK) st = rows_map(&tv, v_out, 128, n_heads, T);
   if (st != MLA_OK) return st;
   UpParams p{block_row, T, (T + 63) / 64, num_blocks};
   cudaError_t e = prefill_attrs();
   if (e == cudaSuccess) {
-    e = launch_pdl(up_proj_kernel, dim3(2, n_heads, (T + kTile - 1) / kTile), dim3(128),
-                   1024 + kUpStages * kUpStageBytes + 256, stream, twk, twv, tpool, tk, tv, p);
+    e = launch_pdl(up_proj_kernel, dim3((T + kTile - 1) / kTile, n_heads), dim3(128), kUpSmem, stream, twk, twv,
+                   tpool, tk, tv, p);
     if (e == cudaSuccess) e = cudaGetLastError();
   }
   if (e != cudaSuccess) return set_error(MLA_ERR_CUDA, "prefill up-projection launch: %s", cudaGetErrorString(e));
@@ -590,8 +610,8 @@ mla_status_t launch_prefill_attn(const void* q_nope, const void* q_rope, const v
                                  const void* kv_pool, const int32_t* block_row, int T, int s, int n_heads,
                                  int num_blocks, float scale, void* out, float* lse, void* stream) {
   CUtensorMap tk, tv, tpool;
-  mla_status_t st = rows_map(&tk, k, 128, n_heads, T, false);
-  if (st == MLA_OK) st = rows_map(&tv, v, 128, n_heads, T, false);
+  mla_status_t st = rows_map(&tk, k, 128, n_heads, T);
+  if (st == MLA_OK) st = rows_map(&tv, v, 128, n_heads, T);
   if (st == MLA_OK) st = pool_map(&tpool, kv_pool, num_blocks);
   if (st != MLA_OK) return st;
   AttParams p{static_cast<const __nv_bfloat16*>(q_nope), static_cast<const __nv_bfloat16*>(q_rope), block_row,
