@@ -11,6 +11,9 @@ selects the others (tiny, v2_4k, varlen, long128k).  Prints ONE JSON line
 (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+  python bench.py --path prefill|upstream|spec [...]   # the NEXT paths, one GPU, each
+      kernel timed alone (spec: the mtp2 batch with --s-q draft tokens as a
+      --draft chain or seeded trees)
 
 Timing: W untimed warm-up steps; then K steps, each bracketed by its own CUDA
 events on the launching stream, with L2 flushed before every step by writing
@@ -66,11 +69,14 @@ def parse_args(argv=None):
                     help="latent cache rows as bf16 (1152 B/token) or E4M3 codes with fp32 block scales "
                          "and a bf16 k_rope (656 B/token)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--path", default="decode", choices=["decode", "prefill", "upstream"],
+    ap.add_argument("--path", default="decode", choices=["decode", "prefill", "upstream", "spec"],
                     help="decode: the absorbed decode step (the headline line); prefill: order-1 prefill of one "
                          "sequence (--prefill T,s); upstream: qkv_a_proj and q_up_absorb for --tokens rows")
     ap.add_argument("--prefill", default="4096,4096", help="T,s of the prefill path (s = T: full prefill)")
     ap.add_argument("--tokens", type=int, default=256, help="token rows of the upstream path")
+    ap.add_argument("--s-q", type=int, default=8, help="draft tokens per sequence of the spec path (1..8)")
+    ap.add_argument("--draft", default="tree", choices=["tree", "chain"],
+                    help="spec path: seeded draft trees (per-query masks) or a chain (the causal rule)")
     return ap.parse_args(argv)
 
 
@@ -619,7 +625,49 @@ def run_next_path(args):
                                          ms_attn, peaks, peak_src),
         }
         ms = ms_up + ms_attn
+        launches = 2 * K
         tokens, workload = s, {"workload": f"prefill T={T} s={s}", "n_heads": H, "pool": "permuted", "seed": 7}
+    elif args.path == "spec":
+        # the mtp2 batch shape (128 sequences, lognormal lengths up to 32K) with
+        # s_q draft tokens per sequence, as a chain (causal) or as seeded trees
+        s_q = args.s_q
+        w = W.preset_workload("mtp2", device=dev, s_q=s_q)
+        tree = args.draft == "tree"
+        dec = mla.Decoder(w.seq_lens, s_q, w.n_heads, w.max_blocks, w.num_blocks, dev, causal=not tree)
+        bt = torch.as_tensor(w.block_table, device=dev)
+        if tree:
+            _, masks_np = W.draft_tree(w.B, s_q, w.meta["seed"])
+            masks = torch.as_tensor(masks_np, device=dev)
+            visible = [int(t) - s_q + bin(int(m)).count("1") for t, row in zip(w.seq_lens, masks_np) for m in row]
+        else:
+            masks = None
+            visible = [int(t) - s_q + 1 + i for t in w.seq_lens for i in range(s_q)]
+        step = lambda: dec.run(w.q_nope, w.q_rope, w.kv_pool, bt, w.w_uk, w.w_uv, draft_masks=masks)
+        step()
+        torch.cuda.synchronize()
+        if dec.status.item() != 0:
+            raise RuntimeError(f"device status {dec.status.item():#x}")
+        if tree:
+            attn = lambda: mla.decode_attn_tree(dec.dims, dec.q_lat, w.q_rope, w.kv_pool, bt, dec.seq_lens_dev, masks,
+                                                dec.plan_dev, dec.num_clusters, dec.o_part, dec.lse_part, dec.o_lat,
+                                                dec.lse, dec.status)
+        else:
+            attn = lambda: mla.decode_attn(dec.dims, dec.q_lat, w.q_rope, w.kv_pool, bt, dec.seq_lens_dev,
+                                           dec.plan_dev, dec.num_clusters, dec.o_part, dec.lse_part, dec.o_lat,
+                                           dec.lse, dec.status)
+        ms_attn = _time_kernel(attn, K, Wm, flush, stream)
+        ms = _time_kernel(step, K, Wm, flush, stream)
+        acc = algorithmic(w.seq_lens, s_q, w.n_heads)
+        flops = sum(visible) * 2 * w.n_heads * (2 * 512 + 64)
+        name = "mla_decode_kernel" + ("<tree>" if tree else "")
+        kern = {name: _roof(flops, acc["attn_bytes"], ms_attn, peaks, peak_src)}
+        tokens = w.B * s_q
+        launches = K * (1 + dec.launches_per_step)
+        T = np.asarray(w.seq_lens)
+        workload = {"workload": f"mtp2 batch, {s_q} draft tokens per sequence as {'seeded trees' if tree else 'a chain'}",
+                    "B": int(w.B), "s_q": s_q, "n_heads": int(w.n_heads), "T_total": int(T.sum()),
+                    "visible_pairs": int(sum(visible)), "seed": w.meta["seed"],
+                    "step": "absorb_q + attention + combine + out_uv, one CUDA-graph replay per step"}
     else:
         N = args.tokens
         g = torch.Generator(device=dev)
@@ -644,13 +692,14 @@ def run_next_path(args):
                                         ms_b, peaks, peak_src),
         }
         ms = ms_a + ms_b
+        launches = 2 * K
         tokens, workload = N, {"workload": f"upstream N={N}", "n_heads": H, "seed": 9}
     return {"metric": f"{args.path} tokens/s (kernels timed one by one)", "value": tokens / (ms * 1e-3),
             "unit": "tokens/s", "n_gpus": 1, "steps": K, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True,
             "dtype": "bf16", "data": "synthetic", "path": args.path,
             "config": dict(workload, l2="flushed before every kernel run (256 MB write; graphs of 10 flush + kernel "
                                         "pairs minus graphs of 10 flushes)"),
-            "kernels": kern, "gpu_launches": 2 * K}
+            "kernels": kern, "gpu_launches": launches}
 
 
 def main(argv=None):

@@ -199,3 +199,19 @@ def preset_workload(name: str, device="cpu", **override) -> Workload:
     w = make_workload(B, s_q, H, seq_lens, seed, pool=pool, device=device, name=name)
     w.meta["lens"] = lens
     return w
+
+
+def draft_tree(B: int, s_q: int, seed: int):
+    """Seeded draft trees for a speculative batch (inputs only): per sequence,
+    the parent of draft i (i >= 1) is drawn uniformly from the committed
+    prefix (-1) and drafts 0 .. i-1, draft 0 hangs off the prefix.  Returns
+    (parents [B][s_q] int, masks int32 [B][s_q]) where bit j of masks[b][i]
+    marks draft j as an ancestor of draft i or draft i itself: the visibility
+    structure a drafter hands to the attention kernel."""
+    rng = np.random.default_rng(seed + 2000)
+    parents = [[-1] + [int(rng.integers(-1, i)) for i in range(1, s_q)] for _ in range(B)]
+    masks = np.zeros((B, s_q), dtype=np.int32)
+    for b, par in enumerate(parents):
+        for i, pa in enumerate(par):
+            masks[b, i] = (1 << i) | (masks[b, pa] if pa >= 0 else 0)
+    return parents, masks

@@ -55,3 +55,21 @@ def test_next_path_roofline_picks_the_binding_unit():
     assert r["bound"] == "tensor" and abs(r["achieved"] - 775.0) < 1e-6 and abs(r["frac"] - 775.0 / 1630.1) < 1e-9
     r = bench._roof(1e6, 30.3e6, 0.010, peaks, "measured")
     assert r["bound"] == "hbm" and abs(r["achieved"] - 3030.0) < 1e-6
+
+
+def test_draft_tree_inputs_are_ancestor_masks():
+    # the spec path's seeded trees: every mask is the oracle's visibility set of its parents
+    parents, masks = W.draft_tree(6, 8, 4)
+    assert masks.dtype == np.int32 and masks.shape == (6, 8)
+    for b in range(6):
+        assert parents[b][0] == -1 and all(-1 <= p < i for i, p in enumerate(parents[b]))
+        assert [int(m) for m in masks[b]] == O.tree_masks(parents[b])
+    # a different seed draws other trees; the same seed the same ones
+    assert W.draft_tree(6, 8, 4)[0] == parents and W.draft_tree(6, 8, 5)[0] != parents
+
+
+def test_spec_path_arguments():
+    a = bench.parse_args(["--path", "spec", "--s-q", "4", "--draft", "chain"])
+    assert (a.path, a.s_q, a.draft) == ("spec", 4, "chain")
+    a = bench.parse_args(["--path", "spec"])
+    assert (a.s_q, a.draft) == (8, "tree")
