@@ -105,6 +105,18 @@ def algorithmic(seq_lens, s_q, H, causal=True, weight_bytes=2, cache_row_bytes=1
                 step_flops=attn_flops + bmm_flops, attn_bytes=attn_bytes, attn_flops=attn_flops)
 
 
+def visible_keys(seq_lens, s_q, masks=None):
+    """Keys each query row attends to, row order (b, i): the T - s_q committed
+    tokens plus, for draft i, the drafts its mask marks (bit j: draft j), or
+    under the causal rule drafts 0..i."""
+    out = []
+    for b, t in enumerate(seq_lens):
+        for i in range(s_q):
+            drafts = bin(int(masks[b][i]) & ((1 << s_q) - 1)).count("1") if masks is not None else i + 1
+            out.append(int(t) - s_q + drafts)
+    return out
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -638,10 +650,9 @@ def run_next_path(args):
         if tree:
             _, masks_np = W.draft_tree(w.B, s_q, w.meta["seed"])
             masks = torch.as_tensor(masks_np, device=dev)
-            visible = [int(t) - s_q + bin(int(m)).count("1") for t, row in zip(w.seq_lens, masks_np) for m in row]
         else:
-            masks = None
-            visible = [int(t) - s_q + 1 + i for t in w.seq_lens for i in range(s_q)]
+            masks_np, masks = None, None
+        visible = visible_keys(w.seq_lens, s_q, masks_np)
         step = lambda: dec.run(w.q_nope, w.q_rope, w.kv_pool, bt, w.w_uk, w.w_uv, draft_masks=masks)
         step()
         torch.cuda.synchronize()

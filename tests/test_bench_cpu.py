@@ -73,3 +73,20 @@ def test_spec_path_arguments():
     assert (a.path, a.s_q, a.draft) == ("spec", 4, "chain")
     a = bench.parse_args(["--path", "spec"])
     assert (a.s_q, a.draft) == (8, "tree")
+
+
+def test_visible_keys_count_the_oracle_visibility():
+    # the spec path's FLOP count: per query row, the keys the oracle's mask keeps
+    parents, masks = W.draft_tree(3, 5, 11)
+    lens = [5, 9, 70]
+    got = bench.visible_keys(lens, 5, masks)
+    want = []
+    for b, T in enumerate(lens):
+        for i in range(5):
+            keep = [t < T - 5 or (masks[b][i] >> (t - (T - 5))) & 1 for t in range(T)]
+            want.append(int(sum(bool(k) for k in keep)))
+    assert got == want
+    # a chain is the causal rule, and the causal count is what algorithmic() charges
+    chain = np.array([O.tree_masks([-1, 0, 1, 2, 3])] * 3, dtype=np.int32)
+    assert bench.visible_keys(lens, 5, chain) == bench.visible_keys(lens, 5)
+    assert sum(bench.visible_keys(lens, 5)) == bench.algorithmic(lens, 5, 16)["pairs"]
