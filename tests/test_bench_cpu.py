@@ -1,6 +1,8 @@
 """CPU pieces of bench.py: the fairer float32 absorbed-order CPU figure computes
 the same attention as the oracle, and the algorithmic accounting matches the
 formulas the measurement uses."""
+import json
+
 import numpy as np
 
 import bench
@@ -90,3 +92,24 @@ def test_visible_keys_count_the_oracle_visibility():
     chain = np.array([O.tree_masks([-1, 0, 1, 2, 3])] * 3, dtype=np.int32)
     assert bench.visible_keys(lens, 5, chain) == bench.visible_keys(lens, 5)
     assert sum(bench.visible_keys(lens, 5)) == bench.algorithmic(lens, 5, 16)["pairs"]
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    # the reference arm times the oracle on the host: one JSON line on rank 0
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    bench.main(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "1"])
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"]
+    assert d["config"]["workload"] == "tiny" and d["steps"] == 2 and d["n_gpus"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_print_nothing(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "1"])
+    assert capsys.readouterr().out.strip() == ""
