@@ -19,11 +19,12 @@ Timing: W untimed warm-up steps; then K steps, each bracketed by its own CUDA
 events on the launching stream, with L2 flushed before every step by writing
 a 256 MB buffer (outside the events); the K-step region is bracketed by a
 barrier and torch.cuda.synchronize() on both sides; ms_per_step is the mean
-per-step event time, max over ranks.  The attention kernel alone is timed the
-same way for the roofline.  `e2e` repeats the step through the public
-mla.GraphedStep API: the step's inputs (queries, page table) copied from
-pinned host memory, the kernels, and the output copied back to pinned host
-memory, all inside the timed region.
+per-step event time, max over ranks.  The attention kernel alone is timed for
+the roofline first in the region, as a short burst (3 replays of a CUDA graph
+of 10 flush + kernel pairs, minus the flushes).  `e2e` repeats the step
+through the public mla.GraphedStep API: the step's inputs (queries, page
+table) copied from pinned host memory, the kernels, and the output copied back
+to pinned host memory, all inside the timed region.
 
 Multi-GPU (torchrun, one process per GPU): data-parallel replicas.  Each rank
 decodes its own batch of the same shape (weak scaling); no collective runs on
@@ -203,12 +204,23 @@ class ClockSampler:
             self.t.join()
             self._sample()
 
-    def summary(self):
+    def mark(self) -> int:
+        """Index of the next sample: segments of the timed region are [mark, next mark)."""
+        return len(self.samples)
+
+    def summary(self, segments=None):
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
-                "samples": len(self.samples), "reasons": names}
+        out = {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+               "samples": len(self.samples), "reasons": names}
+        if segments:
+            seg = {}
+            for name, (a, b) in segments.items():
+                xs = self.samples[a:b]
+                seg[name] = {"sm_mhz": float(statistics.median(xs)) if xs else None, "samples": len(xs)}
+            out["segments"] = seg
+        return out
 
 
 # ----------------------------------------------------------------------------- CPU oracle sample
@@ -402,7 +414,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             for _ in range(10):
                 flush.zero_()
     torch.cuda.synchronize()
-    R = max(3, (K + 9) // 10)
+    # The attention kernel alone is timed as a short burst at the start of the
+    # region, like the measured bf16 peak (best of 10 cuBLAS GEMMs): in a loop of
+    # 200 launches on a B200 it ran into the power cap (SM clock median 1.66 GHz
+    # against 1.97); the per-segment clocks in the line show what each part saw.
+    R = 3
     ea = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(R)]
     ef = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(R)]
     try:
@@ -413,11 +429,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     barrier()
     t_wall = time.perf_counter()
     with sampler:
-        for i in range(K):
-            flush.zero_()
-            ev[i][0].record(stream)
-            run_step()
-            ev[i][1].record(stream)
+        m0 = sampler.mark()
         for i in range(R):
             ea[i][0].record(stream)
             g_attn.replay()
@@ -425,6 +437,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             ef[i][0].record(stream)
             g_flush.replay()
             ef[i][1].record(stream)
+        torch.cuda.synchronize()   # the samples after this point belong to the step loop
+        m1 = sampler.mark()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            run_step()
+            ev[i][1].record(stream)
         barrier()
     t_wall = time.perf_counter() - t_wall
     step_ms = [a.elapsed_time(b) for a, b in ev]
@@ -526,7 +545,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "ms_per_step_percentiles": step_pct,
         "attention_ms_percentiles": attn_pct,
         "attention_timing": f"{R} replays each of a CUDA graph of 10 (L2 flush, attention) pairs and of one of "
-                            "10 flushes; per launch = (pair graph - flush graph) / 10",
+                            "10 flushes, first in the timed region (a burst, like the peak's GEMMs); per launch = "
+                            "(pair graph - flush graph) / 10",
         "roofline": roof,
         "e2e": {"value": tokens / (e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e,
@@ -537,7 +557,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                "before each step",
                 "matches_device_output": e2e_check},
         "gpu_launches": K * dec.launches_per_step + 10 * R,
-        "clocks": sampler.summary(),
+        "clocks": sampler.summary({"attention": (m0, m1), "steps": (m1, None)}),
         "device_status": status,
         "wall_s_timed_region": t_wall,
     }

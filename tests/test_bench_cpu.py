@@ -113,3 +113,11 @@ def test_reference_arm_other_ranks_print_nothing(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     bench.main(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "1"])
     assert capsys.readouterr().out.strip() == ""
+
+
+def test_clock_summary_segments():
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.ok, cs.samples, cs.reasons, cs.max_mhz = True, [1965, 1965, 1900, 1800, 1700], 0x4, 1965
+    out = cs.summary({"steps": (0, 2), "attention": (2, None)})
+    assert out["sm_mhz"] == 1900 and out["reasons"] == ["sw_power_cap"]
+    assert out["segments"] == {"steps": {"sm_mhz": 1965.0, "samples": 2}, "attention": {"sm_mhz": 1800.0, "samples": 3}}
