@@ -135,6 +135,27 @@ def test_plan_random_covers_every_page_once(seed):
     assert buf[11] * 4 <= pb and ns * 128 * 512 * 4 <= ob and ns * 128 * 4 <= lb
 
 
+@pytest.mark.parametrize("seed", range(4))
+def test_non_causal_plan_covers_every_page_of_every_row(seed):
+    # the draft-tree entry point runs non-causal plans: every query row spans its
+    # sequence's whole length (the masks then pick the drafts)
+    rng = np.random.default_rng(100 + seed)
+    B = int(rng.integers(1, 30))
+    s_q = int(rng.integers(1, 9))
+    lens = rng.integers(s_q, 12000, size=B).tolist()
+    C = int(rng.integers(1, 160))
+    dims = mla.make_dims(B, s_q, 128, max(-(-t // 64) for t in lens), 10 ** 6, causal=False)
+    buf, ns = mla.plan(dims, lens, C)
+    cl, items, rows = _unpack(buf)
+    assert (cl, items, rows) == py_plan(lens, s_q, False, 128, C)
+    covered = set()
+    for w in items:
+        b, qi, p0, p1, kv, slot, n = w[:7]
+        assert kv == lens[b] and n == b * s_q + qi
+        covered.update((n, p) for p in range(p0, p1))
+    assert covered == {(b * s_q + i, p) for b in range(B) for i in range(s_q) for p in range(-(-lens[b] // 64))}
+
+
 # ------------------------------------------------------------------ validation (no GPU needed)
 def test_invalid_arguments_return_codes():
     good = mla.make_dims(2, 1, 16, 4, 8)
